@@ -1,0 +1,126 @@
+"""The pins must catch plausible mistakes in the oracle.
+
+Each mutant is a textual edit of a temporary copy of ``oracle/moe_oracle.c``
+(a swapped comparison, an off-by-one, a dropped term, a wrong sign, index or
+constant), compiled with the oracle's own flags and swapped in for the real
+library while the pin checks run.  Every mutant must fail at least one pin;
+the committed oracle is never modified.
+"""
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import build as obuild
+
+import test_oracle_combine as C
+import test_oracle_fp8 as F
+import test_oracle_layout as L
+
+SRC = open(obuild.SRC).read()
+
+# (name, anchor to search from, old text, new text)
+MUTANTS = [
+    ("tie-break t reversed", "orc_cmp_pair", "return x->t < y->t ? -1 : 1;", "return x->t > y->t ? -1 : 1;"),
+    ("expert key dropped", "orc_cmp_pair", "if (x->e != y->e) return x->e < y->e ? -1 : 1;", ""),
+    ("k order reversed", "orc_cmp_pair", "return x->k < y->k ? -1 : 1;", "return x->k > y->k ? -1 : 1;"),
+    ("inclusive expert offsets", "run = 0;",
+     "expert_offset[e] = (int32_t)run;\n            run += expert_count[e];",
+     "run += expert_count[e];\n            expert_offset[e] = (int32_t)run;"),
+    ("dedup row off by one", "distinct (t, p)", "disp_row[j] = (int32_t)d;", "disp_row[j] = (int32_t)d + 1;"),
+    ("dedup keyed by expert", "distinct (t, p)",
+     "has[(int64_t)pairs[r].t * E_part + pairs[r].p] = 1;",
+     "has[(int64_t)pairs[r].t * E_part + (pairs[r].e % E_part)] = 1;"),
+    ("e4m3 ties away", "orc_round_half_even(float q)", "else if (frac == 0.5f) n += (n & 1);",
+     "else if (frac == 0.5f) n += 1;"),
+    ("e4m3 subnormal quantum", "below 2^-6", "a * 512.0f", "a * 256.0f"),
+    ("e4m3 no saturation", "static uint8_t orc_e4m3", "if (E > 8 || code > 0x7E) code = 0x7E;", ""),
+    ("scale constant", "orc_quantize_block", "amax / 448.0f", "amax / 240.0f"),
+    ("bf16 ties away", "orc_f32_to_bf16(float f)", "u += 0x7FFFu + lsb;", "u += 0x8000u;"),
+    ("combine drops last k", "int oracle_combine", "for (int32_t k = 0; k < topk; ++k)",
+     "for (int32_t k = 0; k < topk - 1; ++k)"),
+    ("combine gate index", "int oracle_combine", "float wk = w[t * topk + k];",
+     "float wk = w[t * topk + (topk - 1 - k)];"),
+    ("combine gate sign", "int oracle_combine", "acc[c] = fmaf(wk,", "acc[c] = fmaf(-wk,"),
+    ("combine token row", "int oracle_combine", "y + (int64_t)r * N", "y + (int64_t)t * N"),
+    ("dispatch wrong row", "void oracle_dispatch", "x + (int64_t)disp_token[r] * N", "x + (int64_t)r * N"),
+]
+
+
+def _mutate(anchor, old, new):
+    i = SRC.index(anchor)
+    j = SRC.index(old, i)
+    return SRC[:j] + new + SRC[j + len(old):]
+
+
+def _pins():
+    """A quick cross-section of the oracle's pins."""
+    return [
+        lambda: L.test_layout_exhaustive_tiny(2, 2, 3, 2, (), False),
+        lambda: L.test_layout_exhaustive_tiny(2, 2, 3, 2, (), True),
+        lambda: L.test_layout_exhaustive_tiny(1, 3, 4, 2, (), False),
+        lambda: L.test_layout_invariants(37, 3, 10, 4, True),
+        lambda: F.test_e4m3_exhaustive_vs_table(1.0),
+        lambda: F.test_e4m3_exhaustive_vs_table(2.0 ** 20),
+        F.test_e4m3_saturation_and_signs,
+        F.test_bf16_round_vs_torch,
+        F.test_fp8_dispatch_scales_and_roundtrip,
+        F.test_bf16_dispatch_identity,
+        lambda: C.test_combine_one_hot_identity(3),
+        lambda: C.test_combine_uniform_gates_identity(4),
+        lambda: C.test_combine_within_fp64_bound(5),
+    ]
+
+
+def _load(src, tmp_path, tag):
+    c = tmp_path / f"mut_{tag}.c"
+    so = tmp_path / f"mut_{tag}.so"
+    c.write_text(src)
+    cmd = ["gcc", *obuild.CFLAGS, str(c), "-o", str(so), "-lm"]
+    subprocess.run(cmd, check=True, capture_output=True)
+    return str(so)
+
+
+def _swap(path):
+    """Point the oracle module at another build of the same source."""
+    saved = oracle._lib
+    oracle._lib = None
+    real = obuild.build
+    obuild.build = lambda *a, **k: path
+    try:
+        oracle.lib()
+    finally:
+        obuild.build = real
+    return saved
+
+
+@pytest.mark.parametrize("name,anchor,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_mutant_is_caught(name, anchor, old, new, tmp_path):
+    src = _mutate(anchor, old, new)
+    assert src != SRC
+    path = _load(src, tmp_path, abs(hash(name)) % 10 ** 8)
+    saved = _swap(path)
+    try:
+        caught = 0
+        for pin in _pins():
+            try:
+                pin()
+            except AssertionError:
+                caught += 1
+                break
+        assert caught, f"no pin caught mutant {name!r}"
+    finally:
+        oracle._lib = saved
+
+
+def test_unmutated_copy_passes(tmp_path):
+    path = _load(SRC, tmp_path, "same")
+    saved = _swap(path)
+    try:
+        for pin in _pins():
+            pin()
+    finally:
+        oracle._lib = saved
