@@ -1,0 +1,458 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE dispatch / combine path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+One step = one pass of the whole path over one batch: routing layout ->
+dispatch permute -> combine (libmoe_layout.so, through its C ABI), on the
+M = 4096, N = 7168, G = 256, topk = 8, E_part = 8, Zipf(1.1) workload by
+default.  Inputs are resident in HBM when the timed region starts.  Each
+step is one CUDA-graph replay with events between its kernels; L2 is
+flushed between steps (256 MiB written, then 256 MiB read, untimed).
+
+Printed (rank 0, one JSON line): value = algorithmic HBM bytes of the whole
+path per second (GB/s) over all ranks; tokens/s; per-kernel times; the
+roofline of the dominant kernel against the measured copy bandwidth; the
+end-to-end figure through the public API with host buffers (host->device
+copies of the inputs and device->host copy of the output in the timed
+region); the CPU oracle timed on the host (rank 0, N = 1).
+
+Multi-GPU: one process per GPU under torchrun; every rank runs its own
+batch (data-parallel replicas, no collective on the data path); the time is
+the max over ranks.  ``--impl reference`` times the CPU oracle instead.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+DEFAULT_WORKLOAD = "M4096-zipf1.1"
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes (HBM traffic the path cannot avoid), per kernel
+# ---------------------------------------------------------------------------
+def algorithmic_bytes(w: W.Workload, R_exp: int, R_disp: int) -> dict:
+    M, N, G, k, E = w.M, w.N, w.G, w.topk, w.E_part
+    layout = 4 * M * k + 4 * G + 4 * M * k + 4 * R_disp + 4 * (2 * G + 2 * E + 2)
+    if w.dedup:
+        layout += 4 * M * E + 4 * R_exp
+    s = 1 if w.fp8 else 2
+    dispatch = 2 * M * N + R_disp * N * s + (4 * R_disp * (N // 128) if w.fp8 else 0)
+    dispatch += 4 * M * (E if w.dedup else k)
+    combine = 2 * R_exp * N + 2 * M * N + 8 * M * k
+    return {"layout": layout, "dispatch": dispatch, "combine": combine}
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def traffic_record(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel's
+    source is unchanged since the capture (else None)."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(p) as f:
+            rec = json.load(f)[f"{kernel}@{workload}"]
+    except Exception:
+        return None
+    src = os.path.join(ROOT, "combine_moe_layout_08_b200", "csrc", rec["source"])
+    try:
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    return float(rec["bytes_per_launch"]) if h == rec["source_sha256_16"] else None
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML polled from a thread; read-only)
+# ---------------------------------------------------------------------------
+REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+           0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+           0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+           0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    def __init__(self, torch_device, period_s=0.005):
+        self.samples, self.reasons = [], 0
+        self.period = period_s
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            import torch
+            uuid = str(torch.cuda.get_device_properties(torch_device).uuid)
+            try:
+                self.h = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid) if not uuid.startswith("GPU-") else uuid)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(torch_device.index or 0)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover - no NVML
+            self.err = str(e)
+
+    def _run(self):
+        nv = self.nv
+        get_r = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(get_r(self.h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "samples": len(self.samples),
+                "reasons": [n for b, n in REASONS.items() if self.reasons & b and b != 0x1]}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (the reference arm and the cpu_baseline leg)
+# ---------------------------------------------------------------------------
+def oracle_step_seconds(w, idx, po, gates, x_bits, y_bits):
+    import oracle
+    t0 = time.perf_counter()
+    lay = oracle.layout(idx, po, w.G, w.E_part, w.dedup)
+    oracle.dispatch(x_bits, lay["disp_token"], w.fp8)
+    oracle.combine(y_bits, gates, lay["exp_row"])
+    return time.perf_counter() - t0, lay
+
+
+def sample_workload(w: W.Workload, tokens: int):
+    """The first ``tokens`` tokens of the workload's batch, all inputs drawn
+    by the same generators (host copies)."""
+    import oracle
+    import torch
+    d = W.make_inputs(w, device="cpu", with_y=False)
+    ws = w.replace(M=tokens)
+    idx = d["topk_idx"][:tokens]
+    gates = d["topk_weights"][:tokens]
+    x_bits = oracle.bf16_bits(d["x"][:tokens])
+    y = W.make_expert_outputs(ws)
+    return ws, idx, d["part_of"], gates, x_bits, oracle.bf16_bits(y)
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    tokens = min(w.M, 512)
+    ws, idx, po, gates, x_bits, y_bits = sample_workload(w, tokens)
+    for _ in range(args.warmup):
+        oracle_step_seconds(ws, idx, po, gates, x_bits, y_bits)
+    times = []
+    lay = None
+    for _ in range(args.steps):
+        t, lay = oracle_step_seconds(ws, idx, po, gates, x_bits, y_bits)
+        times.append(t)
+    total = sum(times)
+    b = algorithmic_bytes(ws, lay["R_exp"], lay["R_disp"])
+    step_bytes = sum(b.values())
+    value = step_bytes * args.steps / total / 1e9
+    sample = f"first {tokens} of {w.M} tokens of {w.name}, full N/G/topk/E_part, one oracle pass per step"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "tokens_per_s": round(tokens * args.steps / total, 1),
+        "config": config_of(w, extra={"sample_tokens": tokens}),
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+METRIC = "dispatch+combine HBM GB/s and tokens/s vs ~8 TB/s roofline at 1 B200"
+
+
+def replica_workload(w: W.Workload, rank: int) -> W.Workload:
+    """Each data-parallel replica draws its own batch of the same shape."""
+    return w.replace(seed=w.seed + rank)
+
+
+def reduce_over_ranks(times, units, device):
+    """Max of ``times`` and sum of ``units`` over the ranks of the default
+    process group (identity without one)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(times, dtype=torch.float64, device=device)
+    u = torch.tensor(units, dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return t.tolist(), u.tolist()
+
+
+def config_of(w, extra=None):
+    c = {"workload": w.name, "M": w.M, "N": w.N, "G": w.G, "topk": w.topk, "E_part": w.E_part,
+         "routing": w.routing, "placement": w.placement, "dedup": w.dedup, "fp8": w.fp8,
+         "seed": w.seed, "parallelism": "replicas (one batch per GPU, no collective)"}
+    if extra:
+        c.update(extra)
+    return c
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+
+    import combine_moe_layout_08_b200 as moe
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}: launch N>1 with torchrun")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
+
+    wr = replica_workload(w, rank)
+    d = W.make_inputs(wr, device=dev)
+    prob = moe.MoEProblem(w.M, w.N, w.G, w.topk, w.E_part, w.dedup, w.fp8)
+    buf = moe.MoEBuffers(prob, dev)
+    idx_h, po_h, g_h = d["topk_idx"], d["part_of"], d["topk_weights"]
+    idx = torch.from_numpy(idx_h).to(dev)
+    po = torch.from_numpy(po_h).to(dev)
+    gates = torch.from_numpy(g_h).to(dev)
+    x, y = d["x"], d["y"]
+    stream = torch.cuda.Stream(dev)
+    flush_w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    def flush():
+        flush_w.zero_()
+        torch.sum(flush_r, out=flush_sink)
+
+    # eager warm-up through the public API, then one graph per step with
+    # external events between the kernels
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            buf.step(idx, po, x, y, gates)
+    stream.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        buf.layout_(idx, po)
+        ev[0].record()
+        buf.dispatch_(x)
+        ev[1].record()
+        buf.combine_(y, gates)
+    R_exp = int(buf.layout.expert_offset[w.G].item())
+    R_disp = int(buf.layout.part_offset[w.E_part].item())
+    status = int(buf.layout.status.item())
+    if status:
+        raise SystemExit(f"layout status {status}")
+    abytes = algorithmic_bytes(wr, R_exp, R_disp)
+    step_bytes = sum(abytes.values())
+
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+
+    def timed_step():
+        with torch.cuda.stream(stream):
+            flush()
+            start.record()
+            graph.replay()
+            end.record()
+        end.synchronize()
+        return (start.elapsed_time(end), start.elapsed_time(ev[0]), ev[0].elapsed_time(ev[1]),
+                ev[1].elapsed_time(end))
+
+    for _ in range(max(args.warmup, 3)):
+        timed_step()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    per = []
+    with ClockSampler(dev) as clk:
+        for _ in range(args.steps):
+            per.append(timed_step())
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    per = np.array(per)                                 # [K, 4] ms
+    total_ms = float(per[:, 0].sum())
+    kern_ms = {"layout": float(per[:, 1].mean()), "dispatch": float(per[:, 2].mean()),
+               "combine": float(per[:, 3].mean())}
+
+    # end to end through the public API with host buffers
+    e2e = run_e2e(args, wr, buf, idx_h, po_h, g_h, x, y, stream, dev, flush, step_bytes)
+
+    # aggregate over ranks: bytes and tokens summed, time = max
+    (max_ms, max_e2e_ms), (all_bytes, all_tokens, all_e2e_bytes) = reduce_over_ranks(
+        [total_ms, e2e["total_ms"]], [step_bytes * args.steps, w.M * args.steps, e2e["bytes"]], dev)
+
+    line = None
+    if rank == 0:
+        peak, peak_kind = measured_peak()
+        dom = max(("dispatch", "combine"), key=lambda k: kern_ms[k])
+        ach = abytes[dom] / (kern_ms[dom] * 1e-3) / 1e9
+        kern_names = {"dispatch": "dispatch_fp8_kernel" if w.fp8 else "dispatch_bf16_kernel",
+                      "combine": "combine_kernel"}
+        src = {"dispatch": "dispatch.cu", "combine": "combine.cu"}
+        line = {
+            "metric": METRIC, "value": round(all_bytes / (max_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(max_ms / args.steps, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f8e4m3+bf16" if w.fp8 else "bf16",
+            "data": "synthetic",
+            "tokens_per_s": round(all_tokens / (max_ms * 1e-3), 1),
+            "config": config_of(w, extra={
+                "R_exp": R_exp, "R_disp": R_disp,
+                "l2": "flushed between timed steps (256 MiB write + 256 MiB read, untimed)",
+                "timing": "one CUDA graph replay per step; CUDA events on the launch stream"}),
+            "kernels_us": {k: round(v * 1e3, 2) for k, v in kern_ms.items()},
+            "kernels_gbs": {k: round(abytes[k] / (kern_ms[k] * 1e-3) / 1e9, 1) for k in kern_ms},
+            "algorithmic_bytes_per_step": abytes,
+            "roofline": {"bound": "hbm", "kernel": kern_names[dom], "achieved": round(ach, 1),
+                         "peak": peak, "unit": "GB/s", "frac": round(ach / peak, 4),
+                         "peak_kind": f"of {peak_kind}",
+                         "traffic": traffic_record(kern_names[dom] + "|" + src[dom], w.name)},
+            "frac_of_8tbs": {k: round(abytes[k] / (kern_ms[k] * 1e-3) / 8e12, 4) for k in
+                             ("dispatch", "combine")},
+            "e2e": {"value": round(all_e2e_bytes / (max_e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                    "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                    "tokens_per_s": round(w.M * world * e2e["steps"] / (max_e2e_ms * 1e-3), 1),
+                    "steps": e2e["steps"]},
+            "gpu_launches": 4 * args.steps,
+            "clocks": clk.summary(),
+        }
+    graph.reset()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wr, buf, idx_h, po_h, g_h, x, y)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_e2e(args, w, buf, idx_h, po_h, g_h, x, y, stream, dev, flush, step_bytes):
+    """Public-API calls on host inputs: pinned host -> device copies of every
+    input, layout / dispatch / combine, device -> host copy of the output."""
+    import torch
+    hx = x.cpu().pin_memory()
+    hy = y.cpu().pin_memory()
+    hidx = torch.from_numpy(idx_h).pin_memory()
+    hpo = torch.from_numpy(po_h).pin_memory()
+    hg = torch.from_numpy(g_h).pin_memory()
+    hout = torch.empty(buf.out.shape, dtype=buf.out.dtype).pin_memory()
+    d_idx = torch.empty_like(hidx, device=dev)
+    d_po = torch.empty_like(hpo, device=dev)
+    d_g = torch.empty_like(hg, device=dev)
+    d_x = torch.empty_like(x)
+    d_y = torch.empty_like(y)
+    h2d = sum(t.numel() * t.element_size() for t in (hx, hy, hidx, hpo, hg))
+    d2h = hout.numel() * hout.element_size()
+    steps = max(3, min(args.steps, 50))
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    total = 0.0
+    for i in range(steps + 2):
+        with torch.cuda.stream(stream):
+            flush()
+            s.record()
+            for dst, src in ((d_idx, hidx), (d_po, hpo), (d_g, hg), (d_x, hx), (d_y, hy)):
+                dst.copy_(src, non_blocking=True)
+            out = buf.step(d_idx, d_po, d_x, d_y, d_g)
+            hout.copy_(out, non_blocking=True)
+            e.record()
+        e.synchronize()
+        if i >= 2:
+            total += s.elapsed_time(e)
+    if not torch.equal(hout, buf.out.cpu()):
+        raise SystemExit("end-to-end output mismatch")
+    return {"total_ms": total * args.steps / steps, "bytes": step_bytes * args.steps,
+            "h2d": h2d, "d2h": d2h, "steps": steps}
+
+
+def cpu_baseline(w, buf, idx_h, po_h, g_h, x, y, budget_s=10.0):
+    """The oracle as it stands, single-threaded, on the same full problem,
+    repeated until about ``budget_s`` seconds of CPU work."""
+    import oracle
+    xb = oracle.bf16_bits(x)
+    yb = oracle.bf16_bits(y)
+    times = []
+    lay = None
+    while sum(times) < budget_s and len(times) < 50:
+        t, lay = oracle_step_seconds(w, idx_h, po_h, g_h, xb, yb)
+        times.append(t)
+    b = sum(algorithmic_bytes(w, lay["R_exp"], lay["R_disp"]).values())
+    mean = sum(times) / len(times)
+    return {"value": round(b / mean / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "tokens_per_s": round(w.M / mean, 1),
+            "sample": f"full {w.name} problem (M={w.M}), {len(times)} oracle passes, "
+                      f"{sum(times):.1f} s, single thread"}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(W.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    w = W.get(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

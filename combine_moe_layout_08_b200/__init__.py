@@ -1,0 +1,216 @@
+"""B200 (sm_100a) MoE token dispatch / combine.
+
+Python face of libmoe_layout.so, with the C names:
+
+* :func:`moe_layout`   -- routing layout (counts, prefix sums, row indices)
+* :func:`moe_dispatch` -- dispatch permute, optional dedup and FP8 e4m3 cast
+* :func:`moe_combine`  -- gate-weighted, slot-ordered combine
+
+Tensors are passed as device pointers with the current CUDA stream; this
+module checks dtypes, shapes and devices, allocates nothing inside the calls
+and computes nothing itself.  :func:`alloc_layout` and :class:`MoEBuffers`
+are conveniences that allocate caller-side buffers at worst-case capacity.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+from typing import Optional
+
+import torch
+
+from . import _lib
+from ._lib import (MOE_MAX_E_PART, MOE_MAX_G, MOE_MAX_TOPK, MOE_STATUS_BAD_EXPERT,
+                   MOE_STATUS_BAD_PART, MOE_STATUS_BAD_ROW, MoEError)
+
+__all__ = ["MoEProblem", "MoELayout", "MoEBuffers", "MoEError", "alloc_layout",
+           "layout_workspace_size", "moe_layout", "moe_dispatch", "moe_combine",
+           "moe_status_string", "moe_abi_version", "MOE_STATUS_BAD_EXPERT",
+           "MOE_STATUS_BAD_PART", "MOE_STATUS_BAD_ROW", "MOE_MAX_G", "MOE_MAX_E_PART",
+           "MOE_MAX_TOPK"]
+
+
+@dataclasses.dataclass(frozen=True)
+class MoEProblem:
+    M: int
+    N: int
+    G: int
+    topk: int
+    E_part: int
+    dedup: bool = False
+    fp8: bool = False
+
+    def struct(self) -> _lib.ProblemStruct:
+        return _lib.ProblemStruct(self.M, self.N, self.G, self.topk, self.E_part,
+                                  int(bool(self.dedup)), int(bool(self.fp8)))
+
+    @property
+    def capacity(self) -> int:
+        """Receive-buffer rows at worst case (M * topk)."""
+        return self.M * self.topk
+
+
+@dataclasses.dataclass
+class MoELayout:
+    """Device arrays of one layout (int32), see ``moe_layout_t``."""
+    expert_count: torch.Tensor
+    expert_offset: torch.Tensor
+    part_count: torch.Tensor
+    part_offset: torch.Tensor
+    exp_row: torch.Tensor
+    disp_token: torch.Tensor
+    status: torch.Tensor
+    disp_row: Optional[torch.Tensor] = None
+    exp_to_disp: Optional[torch.Tensor] = None
+
+    def struct(self) -> _lib.LayoutStruct:
+        def p(t):
+            return None if t is None else t.data_ptr()
+        return _lib.LayoutStruct(p(self.expert_count), p(self.expert_offset), p(self.part_count),
+                                 p(self.part_offset), p(self.exp_row), p(self.disp_token),
+                                 p(self.disp_row), p(self.exp_to_disp), p(self.status))
+
+
+def moe_abi_version() -> int:
+    return _lib.load().moe_abi_version()
+
+
+def moe_status_string(code: int) -> str:
+    return _lib.load().moe_status_string(code).decode()
+
+
+def layout_workspace_size(prob: MoEProblem) -> int:
+    s = prob.struct()
+    return int(_lib.load().moe_layout_workspace_size(ctypes.byref(s)))
+
+
+def alloc_layout(prob: MoEProblem, device="cuda") -> MoELayout:
+    """Layout arrays at worst-case capacity on ``device`` (uninitialised)."""
+    cap = max(prob.capacity, 1)
+    i32 = dict(dtype=torch.int32, device=device)
+    return MoELayout(
+        expert_count=torch.empty(prob.G, **i32), expert_offset=torch.empty(prob.G + 1, **i32),
+        part_count=torch.empty(prob.E_part, **i32), part_offset=torch.empty(prob.E_part + 1, **i32),
+        exp_row=torch.empty(cap, **i32), disp_token=torch.empty(cap, **i32),
+        status=torch.empty(1, **i32),
+        disp_row=torch.empty(max(prob.M * prob.E_part, 1), **i32) if prob.dedup else None,
+        exp_to_disp=torch.empty(cap, **i32) if prob.dedup else None)
+
+
+def _stream(t: torch.Tensor, stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream(t.device)
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check(t, name, dtype, numel=None, device=None):
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if numel is not None and t.numel() < numel:
+        raise ValueError(f"{name}: needs >= {numel} elements, has {t.numel()}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def _check_layout(prob: MoEProblem, lay: MoELayout, device):
+    cap = prob.capacity
+    _check(lay.expert_count, "expert_count", torch.int32, prob.G, device)
+    _check(lay.expert_offset, "expert_offset", torch.int32, prob.G + 1, device)
+    _check(lay.part_count, "part_count", torch.int32, prob.E_part, device)
+    _check(lay.part_offset, "part_offset", torch.int32, prob.E_part + 1, device)
+    _check(lay.exp_row, "exp_row", torch.int32, cap, device)
+    _check(lay.disp_token, "disp_token", torch.int32, cap, device)
+    _check(lay.status, "status", torch.int32, 1, device)
+    if prob.dedup:
+        _check(lay.disp_row, "disp_row", torch.int32, prob.M * prob.E_part, device)
+        _check(lay.exp_to_disp, "exp_to_disp", torch.int32, cap, device)
+
+
+def moe_layout(prob: MoEProblem, topk_idx: torch.Tensor, part_of: torch.Tensor,
+               lay: MoELayout, workspace: torch.Tensor, stream=None) -> None:
+    """Routing layout of ``topk_idx`` [M, topk] int32 under ``part_of`` [G] int32."""
+    dev = part_of.device
+    _check(topk_idx, "topk_idx", torch.int32, prob.M * prob.topk, dev)
+    _check(part_of, "part_of", torch.int32, prob.G, dev)
+    _check(workspace, "workspace", torch.uint8, None, dev)
+    _check_layout(prob, lay, dev)
+    s, l = prob.struct(), lay.struct()
+    rc = _lib.load().moe_layout(ctypes.byref(s), topk_idx.data_ptr(), part_of.data_ptr(),
+                                ctypes.byref(l), workspace.data_ptr(), workspace.numel(),
+                                _stream(part_of, stream))
+    if rc:
+        raise MoEError("moe_layout", rc)
+
+
+def moe_dispatch(prob: MoEProblem, x: torch.Tensor, lay: MoELayout, recv_x: torch.Tensor,
+                 recv_scale: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Dispatch rows of ``x`` [M, N] bf16 into ``recv_x`` (bf16, or uint8 with fp8)."""
+    dev = x.device
+    cap = prob.capacity
+    _check(x, "x", torch.bfloat16, prob.M * prob.N, dev)
+    _check(recv_x, "recv_x", torch.uint8 if prob.fp8 else torch.bfloat16, cap * prob.N, dev)
+    if prob.fp8:
+        _check(recv_scale, "recv_scale", torch.float32, cap * (prob.N // 128), dev)
+    _check_layout(prob, lay, dev)
+    s, l = prob.struct(), lay.struct()
+    rc = _lib.load().moe_dispatch(ctypes.byref(s), x.data_ptr(), ctypes.byref(l), recv_x.data_ptr(),
+                                  recv_scale.data_ptr() if recv_scale is not None else None,
+                                  _stream(x, stream))
+    if rc:
+        raise MoEError("moe_dispatch", rc)
+
+
+def moe_combine(prob: MoEProblem, y: torch.Tensor, topk_weights: torch.Tensor, lay: MoELayout,
+                out: torch.Tensor, stream=None) -> None:
+    """out [M, N] bf16 = gate-weighted sum of the expert rows ``y`` [M*topk, N] bf16."""
+    dev = y.device
+    _check(y, "y", torch.bfloat16, prob.capacity * prob.N, dev)
+    _check(topk_weights, "topk_weights", torch.float32, prob.M * prob.topk, dev)
+    _check(out, "out", torch.bfloat16, prob.M * prob.N, dev)
+    _check_layout(prob, lay, dev)
+    s, l = prob.struct(), lay.struct()
+    rc = _lib.load().moe_combine(ctypes.byref(s), y.data_ptr(), topk_weights.data_ptr(),
+                                 ctypes.byref(l), out.data_ptr(), _stream(y, stream))
+    if rc:
+        raise MoEError("moe_combine", rc)
+
+
+class MoEBuffers:
+    """Caller-side device buffers of one problem at worst-case capacity, and
+    the three calls of one pass over them (layout -> dispatch -> combine)."""
+
+    def __init__(self, prob: MoEProblem, device="cuda"):
+        self.prob = prob
+        self.device = torch.device(device)
+        cap = max(prob.capacity, 1)
+        self.layout = alloc_layout(prob, self.device)
+        self.workspace = torch.empty(max(layout_workspace_size(prob), 16), dtype=torch.uint8,
+                                     device=self.device)
+        if prob.fp8:
+            self.recv_x = torch.empty((cap, prob.N), dtype=torch.uint8, device=self.device)
+            self.recv_scale = torch.empty((cap, prob.N // 128), dtype=torch.float32, device=self.device)
+        else:
+            self.recv_x = torch.empty((cap, prob.N), dtype=torch.bfloat16, device=self.device)
+            self.recv_scale = None
+        self.out = torch.empty((max(prob.M, 1), prob.N), dtype=torch.bfloat16, device=self.device)
+
+    def layout_(self, topk_idx, part_of, stream=None):
+        moe_layout(self.prob, topk_idx, part_of, self.layout, self.workspace, stream)
+
+    def dispatch_(self, x, stream=None):
+        moe_dispatch(self.prob, x, self.layout, self.recv_x, self.recv_scale, stream)
+
+    def combine_(self, y, topk_weights, stream=None):
+        moe_combine(self.prob, y, topk_weights, self.layout, self.out, stream)
+
+    def step(self, topk_idx, part_of, x, y, topk_weights, stream=None):
+        self.layout_(topk_idx, part_of, stream)
+        self.dispatch_(x, stream)
+        self.combine_(y, topk_weights, stream)
+        return self.out

@@ -1,0 +1,94 @@
+// extern "C" entry points of libmoe_layout.so: argument validation (before
+// any CUDA call, so that a bad call costs nothing on the device) and the
+// launches.  See include/moe_layout.h for the contract of each call.
+#include <cstdint>
+
+#include "moe_internal.h"
+#include "moe_layout.h"
+
+namespace {
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool valid_problem(const moe_problem_t* p) {
+  if (!p) return false;
+  if (p->M < 0 || p->N <= 0 || (p->N % 8) != 0) return false;
+  if (p->G < 1 || p->G > MOE_MAX_G) return false;
+  if (p->topk < 1 || p->topk > MOE_MAX_TOPK) return false;
+  if (p->E_part < 1 || p->E_part > MOE_MAX_E_PART) return false;
+  if ((p->dedup != 0 && p->dedup != 1) || (p->fp8 != 0 && p->fp8 != 1)) return false;
+  if (p->fp8 && (p->N % 128) != 0) return false;
+  if ((int64_t)p->M * p->topk >= ((int64_t)1 << 31)) return false;
+  if ((int64_t)p->M * p->E_part >= ((int64_t)1 << 31)) return false;
+  return true;
+}
+
+// device int32 array: present and 4-byte aligned
+bool arr(const void* q) { return q != nullptr && aligned(q, 4); }
+
+bool valid_layout(const moe_problem_t* p, const moe_layout_t* l) {
+  if (!l) return false;
+  if (!arr(l->expert_count) || !arr(l->expert_offset) || !arr(l->part_count) ||
+      !arr(l->part_offset) || !arr(l->exp_row) || !arr(l->disp_token) || !arr(l->status))
+    return false;
+  if (p->dedup && (!arr(l->disp_row) || !arr(l->exp_to_disp))) return false;
+  return true;
+}
+
+int cuda_rc(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+const char* moe_status_string(int code) {
+  switch (code) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_ARG: return "invalid argument (sizes, null or misaligned pointer)";
+    case MOE_ERR_WORKSPACE: return "workspace missing or smaller than moe_layout_workspace_size()";
+    case MOE_ERR_CUDA: return "CUDA launch failed";
+    default: return "unknown status code";
+  }
+}
+
+size_t moe_layout_workspace_size(const moe_problem_t* prob) {
+  if (!valid_problem(prob)) return 0;
+  return moe::layout_workspace_bytes(*prob);
+}
+
+int moe_layout(const moe_problem_t* prob, const int32_t* topk_idx, const int32_t* part_of,
+               const moe_layout_t* lay, void* workspace, size_t workspace_bytes,
+               moe_stream_t stream) {
+  if (!valid_problem(prob) || !valid_layout(prob, lay)) return MOE_ERR_ARG;
+  if (!arr(part_of) || (prob->M > 0 && !arr(topk_idx))) return MOE_ERR_ARG;
+  const size_t need = moe::layout_workspace_bytes(*prob);
+  if (!workspace || !aligned(workspace, 16) || workspace_bytes < need) return MOE_ERR_WORKSPACE;
+  return cuda_rc(moe::launch_layout(*prob, topk_idx, part_of, *lay, workspace,
+                                    reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int moe_dispatch(const moe_problem_t* prob, const void* x, const moe_layout_t* lay,
+                 void* recv_x, float* recv_scale, moe_stream_t stream) {
+  if (!valid_problem(prob) || !valid_layout(prob, lay)) return MOE_ERR_ARG;
+  if (prob->M > 0) {
+    if (!x || !aligned(x, 16) || !recv_x || !aligned(recv_x, 16)) return MOE_ERR_ARG;
+    if (prob->fp8 && (!recv_scale || !aligned(recv_scale, 16))) return MOE_ERR_ARG;
+  }
+  return cuda_rc(moe::launch_dispatch(*prob, x, *lay, recv_x, recv_scale,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int moe_combine(const moe_problem_t* prob, const void* y, const float* topk_weights,
+                const moe_layout_t* lay, void* out, moe_stream_t stream) {
+  if (!valid_problem(prob) || !valid_layout(prob, lay)) return MOE_ERR_ARG;
+  if (prob->M > 0) {
+    if (!y || !aligned(y, 16) || !out || !aligned(out, 16)) return MOE_ERR_ARG;
+    if (!arr(topk_weights)) return MOE_ERR_ARG;
+  }
+  return cuda_rc(moe::launch_combine(*prob, y, topk_weights, *lay, out,
+                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

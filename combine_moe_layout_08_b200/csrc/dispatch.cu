@@ -1,0 +1,223 @@
+// Dispatch permute: every token row is read from HBM once and written to each
+// dispatch row that holds it -- topk rows without dedup, one row per
+// partition with dedup.  The all_to_all_kernel of the Triton-distributed
+// issue #117 moves data_src rows into data_dst with optional per-row scales
+// (WITH_SCALE); here the destinations are partitions of one receive buffer
+// in this GPU's HBM.
+//
+// bf16: 16-byte vector loads (non-coherent, no L1 allocation) of the whole
+// row segment into registers, then 16-byte stores to each destination.
+//
+// fp8: the same read, then per 128-column block amax (8 lanes, 16 columns
+// each, reduced with shuffles), scale = amax / 448 (IEEE division), each
+// value divided by the scale (IEEE division) and cast to e4m3 with the
+// saturating round-to-nearest-even conversion; the 16 bytes of a lane are
+// stored to every destination and one lane of the 8 writes the block's
+// scale.  The quantisation is done once per token, not once per copy.
+#include <cuda_fp8.h>
+
+#include <algorithm>
+
+#include "moe_device.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kDThreads = 128;
+constexpr int kMaxDest = MOE_MAX_E_PART > MOE_MAX_TOPK ? MOE_MAX_E_PART : MOE_MAX_TOPK;
+
+struct DispatchArgs {
+  const uint4* __restrict__ x;  // [M][N8]
+  int N8;                       // 16-byte chunks per bf16 row (N / 8)
+  int topk, E, dedup;
+  int cap;                      // receive capacity in rows (M * topk)
+  const int* exp_row;           // [M][topk]
+  const int* disp_row;          // [M][E], dedup only
+  void* recv;                   // [cap][N] bf16 or u8
+  float* recv_scale;            // [cap][N / 128], fp8 only
+  int* status;
+};
+
+// Destination rows of token t, in slot (or partition) order, into smem.
+__device__ __forceinline__ int destinations(const DispatchArgs& a, int t, int* dst, int* nd) {
+  if (warp_id() == 0) {
+    const int lane = lane_id();
+    const int n_ent = a.dedup ? a.E : a.topk;
+    const int* ent = a.dedup ? a.disp_row + (size_t)t * a.E : a.exp_row + (size_t)t * a.topk;
+    int count = 0;
+    bool bad = false;
+    for (int base = 0; base < n_ent; base += kWarp) {
+      const int i = base + lane;
+      const int r = i < n_ent ? ld_nc_i32(ent + i) : -1;
+      const bool ok = r >= 0 && r < a.cap;
+      bad |= (r < -1) || (r >= a.cap);
+      const unsigned bal = __ballot_sync(kFull, ok);
+      if (ok) dst[count + __popc(bal & lanemask_lt())] = r;
+      count += __popc(bal);
+    }
+    if (lane == 0) *nd = count;
+    if (bad) raise_status(a.status, MOE_STATUS_BAD_ROW);
+  }
+  __syncthreads();
+  return *nd;
+}
+
+template <int U>
+__global__ void __launch_bounds__(kDThreads) dispatch_bf16_kernel(DispatchArgs a) {
+  __shared__ int dst[kMaxDest];
+  __shared__ int nd;
+  const int t = blockIdx.x;
+  const int c0 = blockIdx.y * (kDThreads * U) + threadIdx.x;
+  const uint4* src = a.x + (size_t)t * a.N8;
+  uint4 v[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int c = c0 + u * kDThreads;
+    if (c < a.N8) v[u] = ld_nc_v4(src + c);
+  }
+  const int n = destinations(a, t, dst, &nd);
+  uint4* recv = static_cast<uint4*>(a.recv);
+  for (int d = 0; d < n; ++d) {
+    uint4* o = recv + (size_t)dst[d] * a.N8;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = c0 + u * kDThreads;
+      if (c < a.N8) st_v4(o + c, v[u]);
+    }
+  }
+}
+
+// 16 bf16 values (two 16-byte chunks) -> 16 e4m3 bytes, given the block scale
+__device__ __forceinline__ uint4 quantize16(const uint4& lo, const uint4& hi, float scale) {
+  const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+  uint32_t q[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f0 = make_float2(__fdiv_rn(bf16_lo(w[2 * i]), scale), __fdiv_rn(bf16_hi(w[2 * i]), scale));
+    const float2 f1 =
+        make_float2(__fdiv_rn(bf16_lo(w[2 * i + 1]), scale), __fdiv_rn(bf16_hi(w[2 * i + 1]), scale));
+    const uint32_t b0 = __nv_cvt_float2_to_fp8x2(f0, __NV_SATFINITE, __NV_E4M3);
+    const uint32_t b1 = __nv_cvt_float2_to_fp8x2(f1, __NV_SATFINITE, __NV_E4M3);
+    q[i] = (b0 & 0xffffu) | (b1 << 16);
+  }
+  return make_uint4(q[0], q[1], q[2], q[3]);
+}
+
+__device__ __forceinline__ float absmax8(const uint4& v) {
+  float m = fabsf(bf16_lo(v.x));
+  m = fmaxf(m, fabsf(bf16_hi(v.x)));
+  m = fmaxf(m, fabsf(bf16_lo(v.y)));
+  m = fmaxf(m, fabsf(bf16_hi(v.y)));
+  m = fmaxf(m, fabsf(bf16_lo(v.z)));
+  m = fmaxf(m, fabsf(bf16_hi(v.z)));
+  m = fmaxf(m, fabsf(bf16_lo(v.w)));
+  m = fmaxf(m, fabsf(bf16_hi(v.w)));
+  return m;
+}
+
+// Each thread owns a 16-column group g; 8 consecutive lanes form one
+// 128-column scale block.  N is a multiple of 128 and kDThreads of 8, so a
+// lane group is either entirely inside the row or entirely past its end.
+template <int U>
+__global__ void __launch_bounds__(kDThreads) dispatch_fp8_kernel(DispatchArgs a) {
+  __shared__ int dst[kMaxDest];
+  __shared__ int nd;
+  const int t = blockIdx.x;
+  const int N16 = a.N8 >> 1;
+  const int g0 = blockIdx.y * (kDThreads * U) + threadIdx.x;
+  const uint4* src = a.x + (size_t)t * a.N8;
+  uint4 lo[U], hi[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int g = g0 + u * kDThreads;
+    if (g < N16) {
+      lo[u] = ld_nc_v4(src + 2 * g);
+      hi[u] = ld_nc_v4(src + 2 * g + 1);
+    } else {
+      lo[u] = make_uint4(0, 0, 0, 0);
+      hi[u] = lo[u];
+    }
+  }
+  const int n = destinations(a, t, dst, &nd);
+  uint4 q[U];
+  float s[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    float m = fmaxf(absmax8(lo[u]), absmax8(hi[u]));
+    m = fmaxf(m, __shfl_xor_sync(kFull, m, 1));
+    m = fmaxf(m, __shfl_xor_sync(kFull, m, 2));
+    m = fmaxf(m, __shfl_xor_sync(kFull, m, 4));
+    if (m == 0.0f) {
+      s[u] = 0.0f;
+      q[u] = make_uint4(0, 0, 0, 0);
+    } else {
+      s[u] = __fdiv_rn(m, 448.0f);
+      q[u] = quantize16(lo[u], hi[u], s[u]);
+    }
+  }
+  uint4* recv = static_cast<uint4*>(a.recv);  // a row is N bytes = N16 chunks
+  const int N128 = N16 >> 3;
+  const bool scale_lane = (threadIdx.x & 7) == 0;
+  for (int d = 0; d < n; ++d) {
+    const size_t r = (size_t)dst[d];
+    uint4* o = recv + r * N16;
+    float* os = a.recv_scale + r * N128;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int g = g0 + u * kDThreads;
+      if (g < N16) {
+        st_v4(o + g, q[u]);
+        if (scale_lane) os[g >> 3] = s[u];
+      }
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_dispatch(const moe_problem_t& p, const void* x, const moe_layout_t& lay,
+                            void* recv_x, float* recv_scale, cudaStream_t stream) {
+  if (p.M == 0) return cudaSuccess;
+  DispatchArgs a;
+  a.x = static_cast<const uint4*>(x);
+  a.N8 = p.N / 8;
+  a.topk = p.topk;
+  a.E = p.E_part;
+  a.dedup = p.dedup;
+  a.cap = p.M * p.topk;
+  a.exp_row = lay.exp_row;
+  a.disp_row = lay.disp_row;
+  a.recv = recv_x;
+  a.recv_scale = recv_scale;
+  a.status = lay.status;
+
+  // U vectors per thread: the whole row in one block up to Umax * 128 units
+  const int units = p.fp8 ? a.N8 / 2 : a.N8;
+  const int Umax = p.fp8 ? 4 : 8;
+  const int U = std::min(Umax, (units + kDThreads - 1) / kDThreads);
+  const int per_block = kDThreads * U;
+  dim3 grid(p.M, (units + per_block - 1) / per_block);
+  if (!p.fp8) {
+    switch (U) {
+      case 1: dispatch_bf16_kernel<1><<<grid, kDThreads, 0, stream>>>(a); break;
+      case 2: dispatch_bf16_kernel<2><<<grid, kDThreads, 0, stream>>>(a); break;
+      case 3: dispatch_bf16_kernel<3><<<grid, kDThreads, 0, stream>>>(a); break;
+      case 4: dispatch_bf16_kernel<4><<<grid, kDThreads, 0, stream>>>(a); break;
+      case 5: dispatch_bf16_kernel<5><<<grid, kDThreads, 0, stream>>>(a); break;
+      case 6: dispatch_bf16_kernel<6><<<grid, kDThreads, 0, stream>>>(a); break;
+      case 7: dispatch_bf16_kernel<7><<<grid, kDThreads, 0, stream>>>(a); break;
+      default: dispatch_bf16_kernel<8><<<grid, kDThreads, 0, stream>>>(a); break;
+    }
+  } else {
+    switch (U) {
+      case 1: dispatch_fp8_kernel<1><<<grid, kDThreads, 0, stream>>>(a); break;
+      case 2: dispatch_fp8_kernel<2><<<grid, kDThreads, 0, stream>>>(a); break;
+      case 3: dispatch_fp8_kernel<3><<<grid, kDThreads, 0, stream>>>(a); break;
+      default: dispatch_fp8_kernel<4><<<grid, kDThreads, 0, stream>>>(a); break;
+    }
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,93 @@
+// Device-side helpers shared by the layout, dispatch and combine kernels.
+// sm_100a only: plain 16-byte vector memory operations with explicit cache
+// hints, warp-synchronous primitives and status bits.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "moe_layout.h"
+
+namespace moe {
+
+constexpr int kWarp = 32;
+constexpr unsigned kFull = 0xffffffffu;
+
+// ---------------------------------------------------------------------------
+// 16-byte global memory operations
+// ---------------------------------------------------------------------------
+
+// Read-only, streaming: the line is not kept in L1 (each token row is read
+// once per kernel).
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+  uint4 v;
+  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "l"(p));
+  return v;
+}
+
+// Read-only gather of a row that another pass of the kernel does not revisit.
+__device__ __forceinline__ uint4 ld_nc_v4_evict_first(const void* p) {
+  uint4 v;
+  asm("ld.global.nc.L1::no_allocate.L2::evict_first.v4.u32 {%0, %1, %2, %3}, [%4];"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "l"(p));
+  return v;
+}
+
+// Store that does not allocate in L1.
+__device__ __forceinline__ void st_v4(void* p, const uint4& v) {
+  asm volatile("st.global.L1::no_allocate.v4.u32 [%0], {%1, %2, %3, %4};"
+               :
+               : "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+// Streaming store (evict-first in L2): output rows nobody re-reads soon.
+__device__ __forceinline__ void st_cs_v4(void* p, const uint4& v) {
+  asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};"
+               :
+               : "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+__device__ __forceinline__ int ld_nc_i32(const int* p) {
+  int v;
+  asm("ld.global.nc.L1::no_allocate.b32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+
+// ---------------------------------------------------------------------------
+// warp helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ unsigned lanemask_lt() {
+  unsigned m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+__device__ __forceinline__ int lane_id() { return threadIdx.x & (kWarp - 1); }
+__device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
+
+// ---------------------------------------------------------------------------
+// bf16 <-> fp32 (bf16 = upper half of binary32)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// two fp32 -> packed bf16x2, each rounded to nearest-even; `lo` in bits 0..15
+__device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// ---------------------------------------------------------------------------
+// status word
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void raise_status(int* status, int bits) {
+  if (bits && status) atomicOr(status, bits);
+}
+
+}  // namespace moe

@@ -1,0 +1,190 @@
+/*
+ * moe_layout.h -- C ABI of the B200 (sm_100a) MoE token dispatch / combine
+ * library, libmoe_layout.so.
+ *
+ * The path: a routing layout built from top-k expert ids and an
+ * expert-to-partition placement map, a dispatch permute that gathers token
+ * rows into partition- and expert-contiguous receive buffers (optionally one
+ * copy per (token, partition) and optionally cast to FP8 e4m3 with one fp32
+ * scale per 128 columns), and a combine that gate-weights and sums the top-k
+ * expert outputs back into token order.  The E_part destination partitions of
+ * an expert-parallel all-to-all are contiguous regions of one receive buffer
+ * in this GPU's memory.
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer argument except `prob` and `lay` (host structs) is a
+ *     DEVICE pointer, owned and allocated by the caller; nothing is allocated,
+ *     freed or kept by the library.  Device buffers must be 16-byte aligned.
+ *   - Calls are asynchronous on `stream` (NULL = legacy default stream) and
+ *     never synchronise with the host or copy device data back to it.  Two
+ *     calls on different streams that share an output race.
+ *   - The return value reports what the host can see before the launch:
+ *     MOE_OK, MOE_ERR_ARG (invalid sizes, null or misaligned pointers),
+ *     MOE_ERR_WORKSPACE (workspace too small) or MOE_ERR_CUDA (a launch
+ *     failed; nothing is retried).  Problems that only the data reveals are
+ *     recorded in the device status word `lay->status` (MOE_STATUS_* bits);
+ *     the kernels never trap or assert, and skip what they cannot process.
+ *   - Row-major layouts throughout.  bf16 is IEEE binary32's upper half.
+ */
+#ifndef MOE_LAYOUT_H
+#define MOE_LAYOUT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream. */
+typedef struct CUstream_st *moe_stream_t;
+
+/* return codes */
+#define MOE_OK 0
+#define MOE_ERR_ARG 1
+#define MOE_ERR_WORKSPACE 2
+#define MOE_ERR_CUDA 3
+
+/* bits of the device status word (lay->status[0]) */
+#define MOE_STATUS_BAD_EXPERT 1 /* a top-k id outside [0, G): that pair is left out   */
+#define MOE_STATUS_BAD_PART 2   /* a placement entry outside [0, E_part): its expert's
+                                   pairs are left out                                   */
+#define MOE_STATUS_BAD_ROW 4    /* dispatch / combine met a row index outside the
+                                   receive capacity M*topk: that copy / term skipped    */
+
+/* limits checked by every entry point */
+#define MOE_MAX_G 1024
+#define MOE_MAX_E_PART 64
+#define MOE_MAX_TOPK 32
+
+/*
+ * Problem sizes, as the all-to-all benchmark of the Triton-distributed issue
+ * #117 ("All2all performance comparison between Triton-distributed and
+ * DeepEP", Benchmark Configuration) poses them:
+ *   M       tokens (>= 0; M = 0 makes every call a no-op)
+ *   N       hidden size, bf16 columns (> 0, multiple of 8; of 128 with fp8)
+ *   G       experts (1..MOE_MAX_G)
+ *   topk    experts per token (1..MOE_MAX_TOPK); M*topk < 2^31
+ *   E_part  destination partitions (1..MOE_MAX_E_PART)
+ *   dedup   0: one dispatch row per routed (token, expert) pair;
+ *           1: one dispatch row per distinct (token, partition) pair
+ *              ("each token is sent to a GPU only once regardless of how many
+ *              of its experts reside there", Zyphra correlated expert
+ *              placement news item)
+ *   fp8     0: dispatch rows are bf16 copies; 1: e4m3 bytes plus one fp32
+ *           scale per 128 columns (the WITH_SCALE / scale_src / scale_dst
+ *           arguments of the issue #117 all_to_all_kernel)
+ */
+typedef struct moe_problem {
+    int32_t M, N, G, topk, E_part;
+    int32_t dedup, fp8;
+} moe_problem_t;
+
+/*
+ * Layout arrays (device, int32, caller-allocated at worst-case capacity so
+ * that no count has to travel back to the host):
+ *   expert_count  [G]        routed pairs per expert
+ *   expert_offset [G+1]      first expert row of each expert; [G] = R_exp.
+ *                            The expert-row space orders the routed pairs by
+ *                            (partition, expert id, token, slot), so each
+ *                            partition's experts are contiguous and each
+ *                            expert's rows are in token order; within a
+ *                            partition the per-expert ends are the `offs`
+ *                            a grouped GEMM consumes (DeepSpeed PR #8180,
+ *                            "Add Triton grouped-GEMM for MoE experts").
+ *   part_count    [E_part]   dispatch rows per partition
+ *   part_offset   [E_part+1] first dispatch row of each partition; [E_part] =
+ *                            R_disp.  This is the scattered-V receive layout
+ *                            of Purlin section 3.1 ("Layouts"): contiguous,
+ *                            variable-sized partitions indexed by destination.
+ *   exp_row       [M*topk]   expert row of pair (t, k), -1 if left out
+ *   disp_token    [M*topk]   token of each dispatch row (first R_disp used)
+ *   disp_row      [M*E_part] dedup only: dispatch row of (t, p) or -1; rows
+ *                            of a partition are in token order.  Ignored
+ *                            (may be NULL) without dedup, where the dispatch
+ *                            rows are the expert rows.
+ *   exp_to_disp   [M*topk]   dedup only: dispatch row holding the token of
+ *                            each expert row (first R_exp used); may be NULL
+ *                            without dedup.
+ *   status        [1]        MOE_STATUS_* bits; written by moe_layout,
+ *                            OR-ed into by moe_dispatch / moe_combine.
+ * Entries beyond R_exp / R_disp are left untouched.
+ */
+typedef struct moe_layout {
+    int32_t *expert_count;
+    int32_t *expert_offset;
+    int32_t *part_count;
+    int32_t *part_offset;
+    int32_t *exp_row;
+    int32_t *disp_token;
+    int32_t *disp_row;
+    int32_t *exp_to_disp;
+    int32_t *status;
+} moe_layout_t;
+
+/* ABI version of this header (bumped on any incompatible change). */
+#define MOE_ABI_VERSION 1
+int moe_abi_version(void);
+
+/* Human-readable text of a return code; never NULL. */
+const char *moe_status_string(int code);
+
+/*
+ * Bytes of device workspace moe_layout needs for `prob` (0 if prob is
+ * invalid).  The workspace holds per-tile expert / partition histograms; it
+ * need not be zeroed and may be reused once the call has completed.
+ */
+size_t moe_layout_workspace_size(const moe_problem_t *prob);
+
+/*
+ * Routing layout.  Split counts and their prefix sums feed an all-to-all
+ * (Triton-distributed issue #117 test snippet: split_send_buf and
+ * send_split_cumsum); here they are built on the device together with the
+ * row index of every routed pair.
+ *   topk_idx  [M, topk] int32  expert ids
+ *   part_of   [G] int32        placement map: partition of each expert
+ *   lay                         output arrays (host struct of device pointers)
+ *   workspace, workspace_bytes  >= moe_layout_workspace_size(prob), 16-B aligned
+ * Deterministic: the same inputs give the same bits on every call.
+ */
+int moe_layout(const moe_problem_t *prob, const int32_t *topk_idx,
+               const int32_t *part_of, const moe_layout_t *lay,
+               void *workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/*
+ * Dispatch permute (issue #117 all_to_all_kernel: data_src -> data_dst with
+ * optional scale_src -> scale_dst).  Each token row of x is read once and
+ * written to every dispatch row that holds it.
+ *   x           [M, N] bf16
+ *   lay         a layout of the same problem (exp_row, or disp_row with dedup)
+ *   recv_x      [M*topk, N] bf16 (fp8 = 0) or uint8 e4m3 (fp8 = 1); rows
+ *               [0, R_disp) are written
+ *   recv_scale  fp8 only: [M*topk, N/128] fp32; block b of row r holds
+ *               scale = amax / 448 of x[t, 128b .. 128b+127] (0 for an
+ *               all-zero block, whose bytes are then 0), and byte j holds
+ *               e4m3(x / scale), nearest-even, saturating at +-448.
+ *               May be NULL with fp8 = 0.
+ */
+int moe_dispatch(const moe_problem_t *prob, const void *x,
+                 const moe_layout_t *lay, void *recv_x, float *recv_scale,
+                 moe_stream_t stream);
+
+/*
+ * Combine: out[t, :] = bf16( sum_k w[t,k] * y[exp_row[t,k], :] ), one owner
+ * per output element, fp32 fused multiply-adds in slot order k = 0..topk-1
+ * starting from +0, one rounding to bf16 (the ordered, exclusively owned
+ * reduction of Purlin section 3.3, "SCORE").  Left-out pairs (exp_row = -1)
+ * contribute nothing.
+ *   y             [M*topk, N] bf16 expert outputs in expert-row space
+ *   topk_weights  [M, topk] fp32 gates
+ *   out           [M, N] bf16
+ */
+int moe_combine(const moe_problem_t *prob, const void *y,
+                const float *topk_weights, const moe_layout_t *lay, void *out,
+                moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_LAYOUT_H */

@@ -1,0 +1,139 @@
+"""The C ABI without a GPU: the library builds and loads, exports every
+function include/moe_layout.h declares, and rejects invalid calls on the host
+before any CUDA call (fake device pointers never reach a kernel: these tests
+skip on a machine with a GPU, where the GPU tests cover the same checks with
+real buffers)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+from combine_moe_layout_08_b200 import _lib, build as libbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_layout.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^[A-Za-z_][\w\s\*]*?\b(moe_\w+)\s*\(", src, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    libbuild.build()
+    return _lib.load()
+
+
+def test_header_declares_the_path():
+    names = declared_functions()
+    for n in ("moe_layout", "moe_dispatch", "moe_combine", "moe_layout_workspace_size",
+              "moe_status_string", "moe_abi_version"):
+        assert n in names
+
+
+def test_exports_every_declared_symbol(L):
+    for n in declared_functions():
+        assert hasattr(L, n), n
+    assert set(declared_functions()) <= set(_lib.SIGNATURES)
+
+
+def test_dynamic_symbol_table():
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (moe_\w+)", out))
+    assert set(declared_functions()) <= exported
+
+
+def test_version_and_strings(L):
+    assert L.moe_abi_version() == 1
+    for c in range(5):
+        assert L.moe_status_string(c)
+
+
+def P(**kw):
+    d = dict(M=128, N=7168, G=256, topk=8, E_part=8, dedup=0, fp8=0)
+    d.update(kw)
+    return _lib.ProblemStruct(**d)
+
+
+def test_workspace_size(L):
+    from combine_moe_layout_08_b200 import _lib as l2  # noqa: F401
+    ws = L.moe_layout_workspace_size(ctypes.byref(P()))
+    assert ws > 0 and ws % 256 == 0
+    big = L.moe_layout_workspace_size(ctypes.byref(P(M=65536, dedup=1)))
+    assert big > ws
+    # per-tile histograms, one tile per SM-sized token slice
+    T = max(64, ((65536 + 147) // 148 + 31) // 32 * 32)
+    nt = (65536 + T - 1) // T
+    assert big == ((nt * (256 + 8 + 1) * 4 + 255) // 256) * 256
+    for bad in (P(N=7), P(G=0), P(G=1025), P(topk=0), P(topk=33), P(E_part=0), P(E_part=65),
+                P(M=-1), P(fp8=1, N=7176), P(dedup=2), P(M=1 << 28, topk=8)):
+        assert L.moe_layout_workspace_size(ctypes.byref(bad)) == 0
+    assert L.moe_layout_workspace_size(None) == 0
+
+
+no_gpu = pytest.mark.skipif(torch.cuda.is_available(), reason="fake pointers only without a GPU")
+
+FAKE = 0x7f0000000000  # never dereferenced: every call below fails validation
+
+
+def fake_layout(**over):
+    f = {n: FAKE + 4096 * i for i, (n, _) in enumerate(_lib.LayoutStruct._fields_)}
+    f.update(over)
+    return _lib.LayoutStruct(**f)
+
+
+@no_gpu
+def test_layout_rejects_bad_arguments(L):
+    ok_ws = L.moe_layout_workspace_size(ctypes.byref(P()))
+    lay = fake_layout()
+    # invalid problems
+    for bad in (P(N=12), P(G=2000), P(topk=40), P(E_part=100), P(fp8=1, N=136)):
+        assert L.moe_layout(ctypes.byref(bad), FAKE, FAKE, ctypes.byref(lay), FAKE, 1 << 30, None) == 1
+    assert L.moe_layout(None, FAKE, FAKE, ctypes.byref(lay), FAKE, ok_ws, None) == 1
+    assert L.moe_layout(ctypes.byref(P()), FAKE, FAKE, None, FAKE, ok_ws, None) == 1
+    # missing / misaligned arrays
+    assert L.moe_layout(ctypes.byref(P()), FAKE, None, ctypes.byref(lay), FAKE, ok_ws, None) == 1
+    assert L.moe_layout(ctypes.byref(P()), FAKE + 2, FAKE, ctypes.byref(lay), FAKE, ok_ws, None) == 1
+    assert L.moe_layout(ctypes.byref(P()), FAKE, FAKE, ctypes.byref(fake_layout(status=None)),
+                        FAKE, ok_ws, None) == 1
+    assert L.moe_layout(ctypes.byref(P()), FAKE, FAKE, ctypes.byref(fake_layout(exp_row=FAKE + 1)),
+                        FAKE, ok_ws, None) == 1
+    # dedup needs disp_row and exp_to_disp
+    assert L.moe_layout(ctypes.byref(P(dedup=1)), FAKE, FAKE, ctypes.byref(fake_layout(disp_row=None)),
+                        FAKE, 1 << 30, None) == 1
+    # workspace
+    assert L.moe_layout(ctypes.byref(P()), FAKE, FAKE, ctypes.byref(lay), FAKE, ok_ws - 1, None) == 2
+    assert L.moe_layout(ctypes.byref(P()), FAKE, FAKE, ctypes.byref(lay), None, ok_ws, None) == 2
+    assert L.moe_layout(ctypes.byref(P()), FAKE, FAKE, ctypes.byref(lay), FAKE + 8, ok_ws, None) == 2
+
+
+@no_gpu
+def test_dispatch_combine_reject_bad_arguments(L):
+    lay = fake_layout()
+    p = ctypes.byref(P())
+    assert L.moe_dispatch(p, None, ctypes.byref(lay), FAKE, None, None) == 1
+    assert L.moe_dispatch(p, FAKE + 8, ctypes.byref(lay), FAKE, None, None) == 1
+    assert L.moe_dispatch(p, FAKE, ctypes.byref(lay), FAKE + 4, None, None) == 1
+    assert L.moe_dispatch(ctypes.byref(P(fp8=1)), FAKE, ctypes.byref(lay), FAKE, None, None) == 1
+    assert L.moe_dispatch(p, FAKE, None, FAKE, None, None) == 1
+    assert L.moe_combine(p, None, FAKE, ctypes.byref(lay), FAKE, None) == 1
+    assert L.moe_combine(p, FAKE, None, ctypes.byref(lay), FAKE, None) == 1
+    assert L.moe_combine(p, FAKE, FAKE + 2, ctypes.byref(lay), FAKE, None) == 1
+    assert L.moe_combine(p, FAKE, FAKE, ctypes.byref(lay), FAKE + 8, None) == 1
+    assert L.moe_combine(ctypes.byref(P(N=0)), FAKE, FAKE, ctypes.byref(lay), FAKE, None) == 1
+
+
+def test_python_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    """No silent fallback: a missing library that cannot be built raises."""
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "absent.so"))
+    import combine_moe_layout_08_b200.build as b
+    monkeypatch.setattr(b, "build", lambda *a, **k: str(tmp_path / "absent.so"))
+    with pytest.raises(RuntimeError):
+        _lib.load()
