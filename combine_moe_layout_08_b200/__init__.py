@@ -20,11 +20,13 @@ from typing import Optional
 import torch
 
 from . import _lib
-from ._lib import (MOE_MAX_E_PART, MOE_MAX_G, MOE_MAX_TOPK, MOE_STATUS_BAD_EXPERT,
+from ._lib import (MOE_MAX_E_PART, MOE_MAX_G, MOE_MAX_TOPK, MOE_STATIC_SCRATCH_BYTES,
+                   MOE_STATUS_BAD_EXPERT,
                    MOE_STATUS_BAD_PART, MOE_STATUS_BAD_ROW, MoEError)
 
 __all__ = ["MoEProblem", "MoELayout", "MoEBuffers", "MoEError", "alloc_layout",
-           "layout_workspace_size", "moe_layout", "moe_dispatch", "moe_combine",
+           "layout_workspace_size", "moe_layout", "moe_layout_static", "moe_dispatch",
+           "moe_combine",
            "moe_status_string", "moe_abi_version", "MOE_STATUS_BAD_EXPERT",
            "MOE_STATUS_BAD_PART", "MOE_STATUS_BAD_ROW", "MOE_MAX_G", "MOE_MAX_E_PART",
            "MOE_MAX_TOPK"]
@@ -146,6 +148,24 @@ def moe_layout(prob: MoEProblem, topk_idx: torch.Tensor, part_of: torch.Tensor,
                                 _stream(part_of, stream))
     if rc:
         raise MoEError("moe_layout", rc)
+
+
+def moe_layout_static(prob: MoEProblem, topk_idx: torch.Tensor, part_of: torch.Tensor,
+                      lay: MoELayout, stream=None) -> None:
+    """moe_layout without a workspace argument, for callers that cannot
+    allocate device memory: the scratch is a fixed device array inside the
+    library (MOE_STATIC_SCRATCH_BYTES), shared by every call.  Calls that
+    overlap on the GPU race on it; the first call on a device must come
+    before any stream capture."""
+    dev = part_of.device
+    _check(topk_idx, "topk_idx", torch.int32, prob.M * prob.topk, dev)
+    _check(part_of, "part_of", torch.int32, prob.G, dev)
+    _check_layout(prob, lay, dev)
+    s, l = prob.struct(), lay.struct()
+    rc = _lib.load().moe_layout_static(ctypes.byref(s), topk_idx.data_ptr(), part_of.data_ptr(),
+                                       ctypes.byref(l), _stream(part_of, stream))
+    if rc:
+        raise MoEError("moe_layout_static", rc)
 
 
 def moe_dispatch(prob: MoEProblem, x: torch.Tensor, lay: MoELayout, recv_x: torch.Tensor,

@@ -25,6 +25,7 @@ MOE_STATUS_BAD_ROW = 4
 MOE_MAX_G = 1024
 MOE_MAX_E_PART = 64
 MOE_MAX_TOPK = 32
+MOE_STATIC_SCRATCH_BYTES = 256 * 1024
 
 
 class ProblemStruct(ctypes.Structure):
@@ -47,6 +48,9 @@ SIGNATURES = {
     "moe_layout": (ctypes.c_int, [ctypes.POINTER(ProblemStruct), ctypes.c_void_p, ctypes.c_void_p,
                                   ctypes.POINTER(LayoutStruct), ctypes.c_void_p, ctypes.c_size_t,
                                   ctypes.c_void_p]),
+    "moe_layout_static": (ctypes.c_int, [ctypes.POINTER(ProblemStruct), ctypes.c_void_p,
+                                         ctypes.c_void_p, ctypes.POINTER(LayoutStruct),
+                                         ctypes.c_void_p]),
     "moe_dispatch": (ctypes.c_int, [ctypes.POINTER(ProblemStruct), ctypes.c_void_p,
                                     ctypes.POINTER(LayoutStruct), ctypes.c_void_p, ctypes.c_void_p,
                                     ctypes.c_void_p]),

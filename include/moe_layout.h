@@ -152,6 +152,31 @@ int moe_layout(const moe_problem_t *prob, const int32_t *topk_idx,
                void *workspace, size_t workspace_bytes, moe_stream_t stream);
 
 /*
+ * Routing layout that allocates nothing -- the same computation and outputs as
+ * moe_layout, for callers that cannot allocate device memory where they route
+ * tokens (code inside a CUDA-graph capture that must not call cudaMalloc,
+ * runtimes whose memory planner hands out no scratch, C hosts without an
+ * allocator).  The pages have no counterpart of this entry point.
+ *   Scratch: a device array of MOE_STATIC_SCRATCH_BYTES compiled into the
+ *   library, held by every GPU that loads it until the process exits.
+ *   Limit: a problem whose moe_layout_workspace_size() exceeds
+ *   MOE_STATIC_SCRATCH_BYTES is rejected with MOE_ERR_WORKSPACE before any
+ *   launch.  The layout uses at most 148 tiles, so every M fits when
+ *   G + E_part <= 441 (G = 256, E_part = 8 always fits); larger G fit only
+ *   for small M.
+ *   The first call on a device looks up the array's device address (one
+ *   cudaGetSymbolAddress with that device current); make it before any
+ *   stream capture.  Every call shares the array: calls whose execution
+ *   overlaps on the GPU (other streams, other threads) race -- serialise them.
+ *   Nothing in the array needs to start at zero.
+ *   Other arguments, errors and results as moe_layout.
+ */
+#define MOE_STATIC_SCRATCH_BYTES (256 * 1024)
+int moe_layout_static(const moe_problem_t *prob, const int32_t *topk_idx,
+                      const int32_t *part_of, const moe_layout_t *lay,
+                      moe_stream_t stream);
+
+/*
  * Dispatch permute (issue #117 all_to_all_kernel: data_src -> data_dst with
  * optional scale_src -> scale_dst).  Each token row of x is read once and
  * written to every dispatch row that holds it.
