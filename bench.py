@@ -8,8 +8,9 @@ One step = one pass of the whole path over one batch: routing layout ->
 dispatch permute -> combine (libmoe_layout.so, through its C ABI), on the
 M = 4096, N = 7168, G = 256, topk = 8, E_part = 8, Zipf(1.1) workload by
 default.  Inputs are resident in HBM when the timed region starts.  Each
-step is one CUDA-graph replay with events between its kernels; L2 is
-flushed between steps (256 MiB written, then 256 MiB read, untimed).
+step is one CUDA-graph replay whose events bracket its kernels on the
+device; L2 is flushed between steps (256 MiB written, then 256 MiB read,
+untimed).
 
 Printed (rank 0, one JSON line): value = algorithmic HBM bytes of the whole
 path per second (GB/s) over all ranks; tokens/s; per-kernel times; the
@@ -280,14 +281,18 @@ def run_ours(args, w):
         for _ in range(3):
             buf.step(idx, po, x, y, gates)
     stream.synchronize()
-    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+    # events inside the graph bracket the step's kernels on the device (the
+    # graph's own launch latency, which back-to-back steps hide, stays out)
+    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
-        buf.layout_(idx, po)
         ev[0].record()
-        buf.dispatch_(x)
+        buf.layout_(idx, po)
         ev[1].record()
+        buf.dispatch_(x)
+        ev[2].record()
         buf.combine_(y, gates)
+        ev[3].record()
     R_exp = int(buf.layout.expert_offset[w.G].item())
     R_disp = int(buf.layout.part_offset[w.E_part].item())
     status = int(buf.layout.status.item())
@@ -296,18 +301,13 @@ def run_ours(args, w):
     abytes = algorithmic_bytes(wr, R_exp, R_disp)
     step_bytes = sum(abytes.values())
 
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
-
     def timed_step():
         with torch.cuda.stream(stream):
             flush()
-            start.record()
             graph.replay()
-            end.record()
-        end.synchronize()
-        return (start.elapsed_time(end), start.elapsed_time(ev[0]), ev[0].elapsed_time(ev[1]),
-                ev[1].elapsed_time(end))
+        stream.synchronize()
+        return (ev[0].elapsed_time(ev[3]), ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2]),
+                ev[2].elapsed_time(ev[3]))
 
     for _ in range(max(args.warmup, 3)):
         timed_step()
@@ -350,7 +350,8 @@ def run_ours(args, w):
             "config": config_of(w, extra={
                 "R_exp": R_exp, "R_disp": R_disp,
                 "l2": "flushed between timed steps (256 MiB write + 256 MiB read, untimed)",
-                "timing": "one CUDA graph replay per step; CUDA events on the launch stream"}),
+                "timing": "one CUDA graph replay per step; CUDA events recorded inside the graph "
+                          "on the launch stream bracket the step's kernels"}),
             "kernels_us": {k: round(v * 1e3, 2) for k, v in kern_ms.items()},
             "kernels_gbs": {k: round(abytes[k] / (kern_ms[k] * 1e-3) / 1e9, 1) for k in kern_ms},
             "algorithmic_bytes_per_step": abytes,
@@ -362,7 +363,8 @@ def run_ours(args, w):
                              ("dispatch", "combine")},
             "e2e": {"value": round(all_e2e_bytes / (max_e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                     "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
-                    "tokens_per_s": round(w.M * world * e2e["steps"] / (max_e2e_ms * 1e-3), 1),
+                    "tokens_per_s": round(w.M * world * args.steps / (max_e2e_ms * 1e-3), 1),
+                    "ms_per_step": round(max_e2e_ms / args.steps, 4),
                     "steps": e2e["steps"]},
             "gpu_launches": 4 * args.steps,
             "clocks": clk.summary(),

@@ -51,31 +51,36 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(s) <= t for s in _inputs())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
+def build(force: bool = False, verbose: bool = False, defines=(), out: str = None) -> str:
+    """Build the library (``out`` and ``defines`` give a variant build
+    elsewhere, e.g. with other compile-time tuning constants)."""
+    target = out or LIB
+    if not force and not defines and out is None and up_to_date():
         return LIB
     nvcc = _nvcc()
-    os.makedirs(BUILD, exist_ok=True)
+    bdir = BUILD if out is None else os.path.join(os.path.dirname(os.path.abspath(out)), "_obj")
+    os.makedirs(bdir, exist_ok=True)
     objs, log = [], []
     for src in sources():
-        obj = os.path.join(BUILD, os.path.basename(src) + ".o")
-        cmd = [nvcc, *ARCH, *NVFLAGS, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
+        obj = os.path.join(bdir, os.path.basename(src) + ".o")
+        cmd = [nvcc, *ARCH, *NVFLAGS, *[f"-D{d}" for d in defines], "-I", INCLUDE, "-I", CSRC,
+               "-c", src, "-o", obj]
         res = subprocess.run(cmd, capture_output=True, text=True)
         log.append(f"$ {' '.join(cmd)}\n{res.stdout}{res.stderr}")
         if res.returncode != 0:
             raise RuntimeError(f"nvcc failed on {src}:\n{res.stderr}")
         objs.append(obj)
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = target + f".tmp{os.getpid()}"
     cmd = [nvcc, *ARCH, "-shared", "-o", tmp, *objs]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         raise RuntimeError(f"link failed:\n{res.stderr}")
-    os.replace(tmp, LIB)
-    with open(os.path.join(BUILD, "ptxas.log"), "w") as f:
+    os.replace(tmp, target)
+    with open(os.path.join(bdir, "ptxas.log"), "w") as f:
         f.write("\n".join(log))
     if verbose:
         print("\n".join(log))
-    return LIB
+    return target
 
 
 if __name__ == "__main__":

@@ -2,11 +2,15 @@
 //
 // Deterministic by construction, as in the SCORE reduction of Purlin
 // (section 3.3, "The Atom"): exclusive ownership -- one thread owns 8
-// consecutive output columns of one token -- and ordered accumulation -- the
-// fp32 fused multiply-adds run in slot order k = 0..topk-1 from +0.  The
-// gathers of all slots are issued before the first accumulation (up to kKG
-// 16-byte loads in flight per thread), so the ordering costs no memory
-// parallelism; one rounding to bf16 at the end.
+// consecutive output columns of one token per vector -- and ordered
+// accumulation -- the fp32 fused multiply-adds run in slot order
+// k = 0..topk-1 from +0, one rounding to bf16 at the end.
+//
+// One block of 128 threads per (token, column slice).  The token's slot rows
+// and gates are read once into shared memory.  A thread owns U 16-byte
+// vectors and gathers KG slots of all of them before the first accumulation
+// (KG * U = 8 loads in flight per thread for any topk: few slots -> more
+// columns per thread), so the fixed order costs no memory parallelism.
 #include <algorithm>
 
 #include "moe_device.cuh"
@@ -16,7 +20,6 @@ namespace moe {
 namespace {
 
 constexpr int kCThreads = 128;
-constexpr int kKG = 8;  // slots gathered per batch
 
 struct CombineArgs {
   const uint4* __restrict__ y;  // [cap][N8]
@@ -38,6 +41,7 @@ __device__ __forceinline__ void fma8(float* acc, float w, const uint4& v) {
   acc[7] = fmaf(w, bf16_hi(v.w), acc[7]);
 }
 
+template <int KG, int U>
 __global__ void __launch_bounds__(kCThreads) combine_kernel(CombineArgs a) {
   __shared__ int rows[MOE_MAX_TOPK];
   __shared__ float wts[MOE_MAX_TOPK];
@@ -51,31 +55,56 @@ __global__ void __launch_bounds__(kCThreads) combine_kernel(CombineArgs a) {
     wts[tid] = __ldg(a.w + (size_t)t * a.topk + tid);
   }
   __syncthreads();
-  const int c = blockIdx.y * kCThreads + tid;
-  if (c >= a.N8) return;
+  const int c0 = blockIdx.y * (kCThreads * U) + tid;
 
-  float acc[8];
+  float acc[U][8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
-  for (int k0 = 0; k0 < a.topk; k0 += kKG) {
-    uint4 v[kKG];
+  for (int u = 0; u < U; ++u)
 #pragma unroll
-    for (int j = 0; j < kKG; ++j) {
+    for (int j = 0; j < 8; ++j) acc[u][j] = 0.0f;
+  for (int k0 = 0; k0 < a.topk; k0 += KG) {
+    uint4 v[U][KG];
+#pragma unroll
+    for (int j = 0; j < KG; ++j) {
       const int k = k0 + j;
-      if (k < a.topk && rows[k] >= 0) v[j] = ld_nc_v4(a.y + (size_t)rows[k] * a.N8 + c);
+      if (k >= a.topk || rows[k] < 0) continue;
+      const uint4* src = a.y + (size_t)rows[k] * a.N8;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int c = c0 + u * kCThreads;
+        if (c < a.N8) v[u][j] = ld_nc_v4(src + c);
+      }
     }
 #pragma unroll
-    for (int j = 0; j < kKG; ++j) {
+    for (int j = 0; j < KG; ++j) {
       const int k = k0 + j;
-      if (k < a.topk && rows[k] >= 0) fma8(acc, wts[k], v[j]);
+      if (k >= a.topk || rows[k] < 0) continue;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int c = c0 + u * kCThreads;
+        if (c < a.N8) fma8(acc[u], wts[k], v[u][j]);
+      }
     }
   }
-  uint4 o;
-  o.x = pack_bf16x2_rn(acc[0], acc[1]);
-  o.y = pack_bf16x2_rn(acc[2], acc[3]);
-  o.z = pack_bf16x2_rn(acc[4], acc[5]);
-  o.w = pack_bf16x2_rn(acc[6], acc[7]);
-  st_v4(a.out + (size_t)t * a.N8 + c, o);
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int c = c0 + u * kCThreads;
+    if (c < a.N8) {
+      uint4 o;
+      o.x = pack_bf16x2_rn(acc[u][0], acc[u][1]);
+      o.y = pack_bf16x2_rn(acc[u][2], acc[u][3]);
+      o.z = pack_bf16x2_rn(acc[u][4], acc[u][5]);
+      o.w = pack_bf16x2_rn(acc[u][6], acc[u][7]);
+      st_v4(a.out + (size_t)t * a.N8 + c, o);
+    }
+  }
+}
+
+template <int KG, int U>
+cudaError_t launch(const CombineArgs& a, int M, cudaStream_t stream) {
+  const dim3 grid(M, (a.N8 + kCThreads * U - 1) / (kCThreads * U));
+  combine_kernel<KG, U><<<grid, kCThreads, 0, stream>>>(a);
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -92,9 +121,11 @@ cudaError_t launch_combine(const moe_problem_t& p, const void* y, const float* w
   a.topk = p.topk;
   a.cap = p.M * p.topk;
   a.status = lay.status;
-  dim3 grid(p.M, (a.N8 + kCThreads - 1) / kCThreads);
-  combine_kernel<<<grid, kCThreads, 0, stream>>>(a);
-  return cudaGetLastError();
+  // KG slots gathered per batch x U vectors per thread = 8 loads in flight
+  if (p.topk >= 5) return launch<8, 1>(a, p.M, stream);
+  if (p.topk >= 3) return launch<4, 2>(a, p.M, stream);
+  if (p.topk == 2) return launch<2, 4>(a, p.M, stream);
+  return launch<1, 8>(a, p.M, stream);
 }
 
 }  // namespace moe

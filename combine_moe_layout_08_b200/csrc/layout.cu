@@ -8,36 +8,66 @@
 // "Layouts").  With dedup a token owns one dispatch row per partition that
 // holds any of its experts (Zyphra news item, correlated expert placement).
 //
-// Two launches, no host round trip:
-//   1. layout_count_kernel: one block per tile of T tokens.  Warp-aggregated
-//      (match.any) shared-memory histogram of the tile's experts, ballot
-//      counts of the tile's (token, partition) pairs, and status flags.
-//   2. layout_rank_kernel: one block per tile.  Every block reduces the
-//      per-tile histograms (a few hundred KB from L2) into totals and its own
-//      tile prefix, orders experts by (partition, id), scans, and ranks its
-//      pairs stably: warp-private counts, an exclusive scan across warps,
-//      then match.any ranks in (token, slot) order.  Block 0 writes the
-//      global counts / offsets / status.
-// The order of every row is fixed by the data, so results are bitwise
-// reproducible.
+// The routed pairs are cut into tiles of consecutive tokens.  A tile's rows
+// of expert e start at  expert_offset[e] + (rows of e in earlier tiles), and
+// inside the tile they are ranked stably in (token, slot) order: each warp
+// counts its contiguous segment into a warp-private histogram, an exclusive
+// scan across warps gives each warp's base, and a ballot match (one vote per key
+// bit) ranks the lanes of a 32-pair chunk.  Everything is fixed by the data, so the result is
+// bitwise reproducible.
+//
+// Two schedules, no host round trip in either:
+//   * up to kClusterItems routed pairs (decode-sized batches): ONE launch of
+//     a cluster of kClusterCTAs blocks.  Each block counts its tile into shared memory,
+//     the blocks exchange their tile histograms through distributed shared
+//     memory between two hardware cluster barriers, and every block finishes
+//     its own tile.  No workspace is touched.
+//   * larger batches: one tile per SM in two launches -- layout_count_kernel
+//     writes per-tile histograms to the workspace, layout_rank_kernel reduces
+//     them (batched 16-byte loads from L2) and ranks its tile.
+// In both, the tile's expert ids are cached in shared memory when they fit.
+#include <cooperative_groups.h>
+
 #include <algorithm>
 
 #include "moe_device.cuh"
 #include "moe_internal.h"
+
+namespace cg = cooperative_groups;
 
 namespace moe {
 namespace {
 
 constexpr int kLThreads = 512;
 constexpr int kLWarps = kLThreads / kWarp;
+constexpr int kClusterCTAs = 8;
+constexpr int kMaxTileItems = 16384;  // tile ids cached in shared memory (64 KB)
+// Compile-time tuning constants: batches of at most MOE_CLUSTER_ITEMS routed
+// pairs take the one-cluster schedule; tiles of the two-launch schedule hold
+// at least MOE_TILE_MIN_TOKENS tokens.
+#ifndef MOE_CLUSTER_ITEMS
+#define MOE_CLUSTER_ITEMS 8192  // measured on B200: one cluster wins only for small batches
+#endif
+#ifndef MOE_TILE_MIN_TOKENS
+#define MOE_TILE_MIN_TOKENS 64
+#endif
+constexpr int kClusterItems = MOE_CLUSTER_ITEMS;
+static_assert(kClusterItems <= kClusterCTAs * kMaxTileItems, "cluster tiles must fit the id cache");
+// width of each half of the column-sum reduction buffer: one slot per thread
+// and 4 columns per slot (>= MOE_MAX_G, the widest matrix reduced)
+constexpr int kRedW = 4 * kLThreads;
+static_assert(kRedW >= MOE_MAX_G, "reduction buffer narrower than the expert count");
 
 struct LayoutArgs {
-  int M, G, topk, E, dedup, T, n_tiles;
+  int M, G, topk, E, dedup;
+  int T;        // tokens per tile
+  int n_tiles;  // tiles (= blocks)
+  int key_cap;  // ids the shared-memory cache holds (0: read from global)
   const int* __restrict__ idx;
   const int* __restrict__ part_of;
-  int* tile_hist;   // [n_tiles][G]
-  int* tile_phist;  // [n_tiles][E], dedup only
-  int* tile_flags;  // [n_tiles]
+  int* tile_hist;   // [n_tiles][G]   (two-launch schedule)
+  int* tile_phist;  // [n_tiles][E]   (two-launch schedule, dedup)
+  int* tile_flags;  // [n_tiles]      (two-launch schedule)
   int* expert_count;
   int* expert_offset;
   int* part_count;
@@ -51,115 +81,183 @@ struct LayoutArgs {
 
 __device__ __forceinline__ bool valid_part(int p, int E) { return p >= 0 && p < E; }
 
-// ---------------------------------------------------------------------------
-// kernel 1: per-tile histograms
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kLThreads) layout_count_kernel(LayoutArgs a) {
-  extern __shared__ int sm[];
-  int* hist = sm;              // [G]
-  int* part_s = hist + a.G;    // [G]
-  int* phist = part_s + a.G;   // [E]
-  __shared__ int flags;
+struct Tile {
+  int t0, ntok, n_items;
+};
 
-  const int tid = threadIdx.x, lane = lane_id(), warp = warp_id();
-  const int b = blockIdx.x;
-  for (int i = tid; i < a.G; i += kLThreads) {
-    hist[i] = 0;
-    part_s[i] = __ldg(a.part_of + i);
-  }
-  for (int i = tid; i < a.E; i += kLThreads) phist[i] = 0;
-  if (tid == 0) flags = 0;
-  __syncthreads();
-
-  int my_flags = 0;
-  if (b == 0) {
-    for (int e = tid; e < a.G; e += kLThreads)
-      if (!valid_part(part_s[e], a.E)) my_flags |= MOE_STATUS_BAD_PART;
-  }
-
-  const int t0 = b * a.T;
-  const int ntok = max(0, min(a.M - t0, a.T));
-  const int n_items = ntok * a.topk;
-  const int* idx = a.idx + (size_t)t0 * a.topk;
-
-  // expert histogram; lanes holding the same expert add once
-  for (int i0 = warp * kWarp; i0 < n_items; i0 += kLThreads) {
-    const int i = i0 + lane;
-    int key = -1;
-    if (i < n_items) {
-      const int e = __ldg(idx + i);
-      if (e < 0 || e >= a.G) {
-        my_flags |= MOE_STATUS_BAD_EXPERT;
-      } else if (valid_part(part_s[e], a.E)) {
-        key = e;
-      }
-    }
-    const unsigned peers = __match_any_sync(kFull, key);
-    if (key >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[key], __popc(peers));
-  }
-
-  // distinct (token, partition) pairs of the tile
-  if (a.dedup) {
-    for (int j0 = warp * kWarp; j0 < ntok; j0 += kLThreads) {
-      const int tl = j0 + lane;
-      unsigned long long mask = 0ull;
-      if (tl < ntok) {
-        for (int k = 0; k < a.topk; ++k) {
-          const int e = __ldg(idx + (size_t)tl * a.topk + k);
-          if (e >= 0 && e < a.G) {
-            const int p = part_s[e];
-            if (valid_part(p, a.E)) mask |= 1ull << p;
-          }
-        }
-      }
-      for (int p = 0; p < a.E; ++p) {
-        const unsigned bal = __ballot_sync(kFull, (mask >> p) & 1ull);
-        if (lane == 0 && bal) atomicAdd(&phist[p], __popc(bal));
-      }
-    }
-  }
-  if (my_flags) atomicOr(&flags, my_flags);
-  __syncthreads();
-
-  int* th = a.tile_hist + (size_t)b * a.G;
-  for (int i = tid; i < a.G; i += kLThreads) th[i] = hist[i];
-  if (a.dedup)
-    for (int i = tid; i < a.E; i += kLThreads) a.tile_phist[(size_t)b * a.E + i] = phist[i];
-  if (tid == 0) a.tile_flags[b] = flags;
+__device__ __forceinline__ Tile tile_of(const LayoutArgs& a, int b) {
+  Tile t;
+  t.t0 = b * a.T;
+  t.ntok = max(0, min(a.M - t.t0, a.T));
+  t.n_items = t.ntok * a.topk;
+  return t;
 }
 
 // ---------------------------------------------------------------------------
-// block-wide building blocks of kernel 2
+// shared-memory plan (ints, every array 16-byte aligned)
+// ---------------------------------------------------------------------------
+struct LayoutSmem {
+  int part_s, tot, pre, eoff, pos, scanbuf, cta_hist, red, whist, ewhist, keycnt, keystart, pc,
+      poff, ptot, ppre, pbase, cta_phist, wp, warp_tot, misc, keys, total;
+  __host__ __device__ static int up4(int x) { return (x + 3) & ~3; }
+  __host__ __device__ LayoutSmem(int G, int E, int key_cap) {
+    const int RW = kRedW;
+    int o = 0;
+    part_s = o; o += up4(G);
+    tot = o; o += up4(G);
+    pre = o; o += up4(G);
+    eoff = o; o += up4(G);
+    pos = o; o += up4(G);
+    scanbuf = o; o += up4(G);
+    cta_hist = o; o += up4(G);
+    red = o; o += up4(2 * RW);
+    whist = o; o += up4(kLWarps * G);
+    ewhist = o; o += up4(kLWarps * (E + 1));
+    keycnt = o; o += up4(E + 1);
+    keystart = o; o += up4(E + 1);
+    pc = o; o += up4(E);
+    poff = o; o += up4(E + 1);
+    ptot = o; o += up4(E);
+    ppre = o; o += up4(E);
+    pbase = o; o += up4(E);
+    cta_phist = o; o += up4(E);
+    wp = o; o += up4(kLWarps * E);
+    warp_tot = o; o += up4(kLWarps);
+    misc = o; o += 4;
+    keys = o; o += up4(key_cap);
+    total = o;
+  }
+};
+
+struct Smem {
+  int *part_s, *tot, *pre, *eoff, *pos, *scanbuf, *cta_hist, *red, *whist, *ewhist, *keycnt,
+      *keystart, *pc, *poff, *ptot, *ppre, *pbase, *cta_phist, *wp, *warp_tot, *misc, *keys;
+  __device__ Smem(int* sm, const LayoutSmem& P)
+      : part_s(sm + P.part_s), tot(sm + P.tot), pre(sm + P.pre), eoff(sm + P.eoff),
+        pos(sm + P.pos), scanbuf(sm + P.scanbuf), cta_hist(sm + P.cta_hist), red(sm + P.red),
+        whist(sm + P.whist), ewhist(sm + P.ewhist), keycnt(sm + P.keycnt),
+        keystart(sm + P.keystart), pc(sm + P.pc), poff(sm + P.poff), ptot(sm + P.ptot),
+        ppre(sm + P.ppre), pbase(sm + P.pbase), cta_phist(sm + P.cta_phist), wp(sm + P.wp),
+        warp_tot(sm + P.warp_tot), misc(sm + P.misc), keys(sm + P.keys) {}
+};
+
+// ---------------------------------------------------------------------------
+// block-wide building blocks
 // ---------------------------------------------------------------------------
 
-// Column sums of a [rows][cols] int matrix in global memory: total over all
-// rows and partial over rows < b.  `red` holds 2 * max(kLThreads, cols) ints.
-__device__ void column_sums(const int* src, int rows, int cols, int b, int* red,
-                            int* total, int* before) {
+// Expert id of tile pair i (shared-memory cache or global).
+struct RawIds {
+  const int* g;  // tile base in global memory
+  const int* s;  // shared-memory cache or nullptr
+  __device__ __forceinline__ int operator()(int i) const { return s ? s[i] : __ldg(g + i); }
+};
+
+// Fill the shared-memory cache of the tile's ids (16-byte loads when aligned),
+// zero the block's scratch and load the placement map.  Ends with a barrier.
+__device__ void stage_tile(const LayoutArgs& a, const Tile& tl, const Smem& S, RawIds& ids) {
   const int tid = threadIdx.x;
-  const int S = cols <= kLThreads ? kLThreads / cols : 1;
-  const int RW = max(kLThreads, cols);
-  for (int slot = tid; slot < cols * S; slot += kLThreads) {
-    const int c = slot % cols, s = slot / cols;
-    int all = 0, bef = 0;
+  const int* src = a.idx + (size_t)tl.t0 * a.topk;
+  ids.g = src;
+  ids.s = nullptr;
+  if (tl.n_items <= a.key_cap) {
+    ids.s = S.keys;
+    const int n = tl.n_items;
+    if ((reinterpret_cast<uintptr_t>(src) & 15) == 0) {
+      const int n4 = n >> 2;
+      const int4* s4 = reinterpret_cast<const int4*>(src);
+      int4* k4 = reinterpret_cast<int4*>(S.keys);
 #pragma unroll 4
-    for (int r = s; r < rows; r += S) {
-      const int v = __ldcg(src + (size_t)r * cols + c);
-      all += v;
-      bef += (r < b) ? v : 0;
+      for (int i = tid; i < n4; i += kLThreads) k4[i] = __ldg(s4 + i);
+      for (int i = (n4 << 2) + tid; i < n; i += kLThreads) S.keys[i] = __ldg(src + i);
+    } else {
+#pragma unroll 4
+      for (int i = tid; i < n; i += kLThreads) S.keys[i] = __ldg(src + i);
     }
-    red[slot] = all;
-    red[RW + slot] = bef;
+  }
+  for (int e = tid; e < a.G; e += kLThreads) S.part_s[e] = __ldg(a.part_of + e);
+  for (int i = tid; i < kLWarps * a.G; i += kLThreads) S.whist[i] = 0;
+  for (int i = tid; i < kLWarps * (a.E + 1); i += kLThreads) S.ewhist[i] = 0;
+  for (int p = tid; p < a.E; p += kLThreads) {
+    S.pc[p] = 0;
+    S.pbase[p] = 0;
+    S.cta_phist[p] = 0;
+  }
+  if (tid < 4) S.misc[tid] = 0;
+  __syncthreads();
+}
+
+// Status bits of the tile (bad expert ids; block `first` also checks the map).
+__device__ int scan_flags(const LayoutArgs& a, const Tile& tl, const Smem& S, const RawIds& ids,
+                          bool first) {
+  int f = 0;
+  for (int i = threadIdx.x; i < tl.n_items; i += kLThreads) {
+    const int e = ids(i);
+    if (e < 0 || e >= a.G) f |= MOE_STATUS_BAD_EXPERT;
+  }
+  if (first)
+    for (int e = threadIdx.x; e < a.G; e += kLThreads)
+      if (!valid_part(S.part_s[e], a.E)) f |= MOE_STATUS_BAD_PART;
+  return f;
+}
+
+// Per-warp counts of the keys of [0, n) (warp w owns the w-th contiguous
+// segment), then an exclusive scan across warps: on return whist[w*K + k]
+// is the number of elements with key k in segments before w, and
+// key_count[k] (if given) the total.  whist must be zero on entry.
+template <class KeyOf>
+__device__ void rank_count(int n, int K, int* whist, int* key_count, KeyOf key_of) {
+  const int lane = lane_id(), warp = warp_id();
+  const int seg = (n + kLWarps - 1) / kLWarps;
+  const int beg = min(n, warp * seg), end = min(n, beg + seg);
+  const int nbits = key_bits(K);
+  int* wh = whist + warp * K;
+  for (int c = beg; c < end; c += kWarp) {
+    const int i = c + lane;
+    const int key = i < end ? key_of(i) : -1;
+    const unsigned peers = match_peers(key, nbits);
+    if (key >= 0 && lane == __ffs(peers) - 1) wh[key] += __popc(peers);
+    __syncwarp();
   }
   __syncthreads();
-  for (int c = tid; c < cols; c += kLThreads) {
-    int all = 0, bef = 0;
-    for (int s = 0; s < S; ++s) {
-      all += red[s * cols + c];
-      bef += red[RW + s * cols + c];
+  for (int key = threadIdx.x; key < K; key += kLThreads) {
+    int v[kLWarps];
+#pragma unroll
+    for (int w = 0; w < kLWarps; ++w) v[w] = whist[w * K + key];
+    int run = 0;
+#pragma unroll
+    for (int w = 0; w < kLWarps; ++w) {
+      whist[w * K + key] = run;
+      run += v[w];
     }
-    total[c] = all;
-    before[c] = bef;
+    if (key_count) key_count[key] = run;
+  }
+  __syncthreads();
+}
+
+// Second pass of the stable rank: on_rank(i, key, rank) with rank = number of
+// elements j < i with the same key; on_skip(i) for keys < 0.
+template <class KeyOf, class OnRank, class OnSkip>
+__device__ void rank_assign(int n, int K, int* whist, KeyOf key_of, OnRank on_rank,
+                            OnSkip on_skip) {
+  const int lane = lane_id(), warp = warp_id();
+  const int seg = (n + kLWarps - 1) / kLWarps;
+  const int beg = min(n, warp * seg), end = min(n, beg + seg);
+  int* wh = whist + warp * K;
+  const unsigned lt = lanemask_lt();
+  const int nbits = key_bits(K);
+  for (int c = beg; c < end; c += kWarp) {
+    const int i = c + lane;
+    const int key = i < end ? key_of(i) : -1;
+    const unsigned peers = match_peers(key, nbits);
+    const int base = key >= 0 ? wh[key] : 0;
+    __syncwarp();
+    if (key >= 0) {
+      on_rank(i, key, base + __popc(peers & lt));
+      if (lane == __ffs(peers) - 1) wh[key] = base + __popc(peers);
+    } else if (i < end) {
+      on_skip(i);
+    }
+    __syncwarp();
   }
   __syncthreads();
 }
@@ -200,257 +298,338 @@ __device__ int block_exclusive_scan(int* data, int n, int* warp_tot) {
   return total;
 }
 
-// Stable counting rank of n elements: rank(i) = number of j < i with the same
-// key.  The elements are cut into kLWarps contiguous segments, one per warp.
-//   key_of(i) -> key in [0, K) or -1 (element skipped: on_skip(i))
-//   on_rank(i, key, rank)
-//   whist: kLWarps * K ints, zero on entry
-//   key_count: [K] totals per key, or nullptr
-template <class KeyOf, class OnRank, class OnSkip>
-__device__ void block_stable_rank(int n, int K, int* whist, int* key_count,
-                                  KeyOf key_of, OnRank on_rank, OnSkip on_skip) {
-  const int lane = lane_id(), warp = warp_id();
-  const int seg = (n + kLWarps - 1) / kLWarps;
-  const int beg = min(n, warp * seg), end = min(n, beg + seg);
-  int* wh = whist + warp * K;
-  for (int c = beg; c < end; c += kWarp) {
-    const int i = c + lane;
-    const int key = i < end ? key_of(i) : -1;
-    const unsigned peers = __match_any_sync(kFull, key);
-    if (key >= 0 && lane == __ffs(peers) - 1) wh[key] += __popc(peers);
-  }
-  __syncthreads();
-  for (int key = threadIdx.x; key < K; key += kLThreads) {
-    int run = 0;
-    for (int w = 0; w < kLWarps; ++w) {
-      const int v = whist[w * K + key];
-      whist[w * K + key] = run;
-      run += v;
+// Partition bit mask of token tl of the tile (valid pairs only).
+__device__ __forceinline__ unsigned long long token_mask(const LayoutArgs& a, const RawIds& ids,
+                                                        const int* part_s, int tl) {
+  unsigned long long mask = 0ull;
+  for (int k = 0; k < a.topk; ++k) {
+    const int e = ids(tl * a.topk + k);
+    if (e >= 0 && e < a.G) {
+      const int p = part_s[e];
+      if (valid_part(p, a.E)) mask |= 1ull << p;
     }
-    if (key_count) key_count[key] = run;
   }
-  __syncthreads();
-  const unsigned lt = lanemask_lt();
-  for (int c = beg; c < end; c += kWarp) {
-    const int i = c + lane;
-    const int key = i < end ? key_of(i) : -1;
-    const unsigned peers = __match_any_sync(kFull, key);
-    const int base = key >= 0 ? wh[key] : 0;
-    __syncwarp();
-    if (key >= 0) {
-      on_rank(i, key, base + __popc(peers & lt));
-      if (lane == __ffs(peers) - 1) wh[key] = base + __popc(peers);
-    } else if (i < end) {
-      on_skip(i);
+  return mask;
+}
+
+// dedup: tokens of the tile holding partition p, into cta_phist[p]
+__device__ void count_tile_parts(const LayoutArgs& a, const Tile& tl, const Smem& S,
+                                 const RawIds& ids) {
+  const int lane = lane_id();
+  for (int r0 = 0; r0 < tl.ntok; r0 += kLThreads) {
+    const int t = r0 + threadIdx.x;
+    const unsigned long long mask = t < tl.ntok ? token_mask(a, ids, S.part_s, t) : 0ull;
+    for (int p = 0; p < a.E; ++p) {
+      const unsigned bal = __ballot_sync(kFull, (mask >> p) & 1ull);
+      if (lane == 0 && bal) atomicAdd(&S.cta_phist[p], __popc(bal));
     }
-    __syncwarp();
   }
   __syncthreads();
 }
 
-// shared-memory plan of kernel 2 (ints)
-struct RankSmem {
-  int part_s, tot, pre, eoff, erank, scanbuf, red, whist, keycnt, keystart, pc, poff, ptot,
-      ppre, pbase, wp, warp_tot, misc, total;
-  __host__ __device__ RankSmem(int G, int E) {
-    const int RW = G > kLThreads ? G : kLThreads;
-    const int KW = G > E + 1 ? G : E + 1;
-    int o = 0;
-    part_s = o; o += G;
-    tot = o; o += G;
-    pre = o; o += G;
-    eoff = o; o += G;
-    erank = o; o += G;
-    scanbuf = o; o += G;
-    red = o; o += 2 * RW;
-    whist = o; o += kLWarps * KW;
-    keycnt = o; o += E + 1;
-    keystart = o; o += E + 1;
-    pc = o; o += E;
-    poff = o; o += E + 1;
-    ptot = o; o += E;
-    ppre = o; o += E;
-    pbase = o; o += E;
-    wp = o; o += kLWarps * E;
-    warp_tot = o; o += kLWarps;
-    misc = o; o += 4;
-    total = o;
-  }
-};
-
-// ---------------------------------------------------------------------------
-// kernel 2: totals, offsets and stable ranks
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kLThreads) layout_rank_kernel(LayoutArgs a) {
-  extern __shared__ int sm[];
-  const int G = a.G, E = a.E, b = blockIdx.x, nt = a.n_tiles;
-  const RankSmem P(G, E);
-  int* part_s = sm + P.part_s;
-  int* tot = sm + P.tot;
-  int* pre = sm + P.pre;
-  int* eoff = sm + P.eoff;
-  int* erank = sm + P.erank;
-  int* scanbuf = sm + P.scanbuf;
-  int* red = sm + P.red;
-  int* whist = sm + P.whist;
-  int* keycnt = sm + P.keycnt;
-  int* keystart = sm + P.keystart;
-  int* pc = sm + P.pc;
-  int* poff = sm + P.poff;
-  int* ptot = sm + P.ptot;
-  int* ppre = sm + P.ppre;
-  int* pbase = sm + P.pbase;
-  int* wp = sm + P.wp;
-  int* warp_tot = sm + P.warp_tot;
-  int* misc = sm + P.misc;
-  const int tid = threadIdx.x, lane = lane_id(), warp = warp_id();
-  const int KW = G > E + 1 ? G : E + 1;
-
-  for (int e = tid; e < G; e += kLThreads) part_s[e] = __ldg(a.part_of + e);
-  for (int i = tid; i < kLWarps * KW; i += kLThreads) whist[i] = 0;
-  for (int p = tid; p < E; p += kLThreads) {
-    pc[p] = 0;
-    pbase[p] = 0;
-  }
-  if (tid == 0) misc[0] = 0;
-  __syncthreads();
-
-  // 1. totals over all tiles and the prefix of the tiles before this one
-  column_sums(a.tile_hist, nt, G, b, red, tot, pre);
-  if (a.dedup) column_sums(a.tile_phist, nt, E, b, red, ptot, ppre);
-
-  // 2. expert order (partition, id); experts of invalid partitions last
+// expert order (partition, id) -> pos[e]; offsets eoff[e], partition counts
+// and offsets.  Needs tot[] (and ptot[] with dedup).  Returns R_exp.
+__device__ int finish_offsets(const LayoutArgs& a, const Smem& S) {
+  const int G = a.G, E = a.E, tid = threadIdx.x;
   auto ekey = [&](int e) {
-    const int p = part_s[e];
+    const int p = S.part_s[e];
     return valid_part(p, E) ? p : E;
   };
-  block_stable_rank(
-      G, E + 1, whist, keycnt, ekey, [&](int e, int, int r) { erank[e] = r; }, [](int) {});
+  rank_count(G, E + 1, S.ewhist, S.keycnt, ekey);
   if (tid == 0) {
     int run = 0;
     for (int k = 0; k <= E; ++k) {
-      keystart[k] = run;
-      run += keycnt[k];
+      S.keystart[k] = run;
+      run += S.keycnt[k];
     }
   }
   __syncthreads();
-  for (int e = tid; e < G; e += kLThreads) {
-    const int pos = keystart[ekey(e)] + erank[e];
-    erank[e] = pos;
-    scanbuf[pos] = tot[e];
-  }
+  rank_assign(
+      G, E + 1, S.ewhist, ekey, [&](int e, int k, int r) { S.pos[e] = S.keystart[k] + r; },
+      [](int) {});
+  for (int e = tid; e < G; e += kLThreads) S.scanbuf[S.pos[e]] = S.tot[e];
   __syncthreads();
-  const int R_exp = block_exclusive_scan(scanbuf, G, warp_tot);
+  const int R_exp = block_exclusive_scan(S.scanbuf, G, S.warp_tot);
   for (int e = tid; e < G; e += kLThreads) {
-    eoff[e] = scanbuf[erank[e]];
-    if (!a.dedup && valid_part(part_s[e], E) && tot[e]) atomicAdd(&pc[part_s[e]], tot[e]);
+    S.eoff[e] = S.scanbuf[S.pos[e]];
+    if (!a.dedup && valid_part(S.part_s[e], E) && S.tot[e]) atomicAdd(&S.pc[S.part_s[e]], S.tot[e]);
   }
   __syncthreads();
   if (tid == 0) {
     int run = 0;
     for (int p = 0; p < E; ++p) {
-      if (a.dedup) pc[p] = ptot[p];
-      poff[p] = run;
-      run += pc[p];
+      if (a.dedup) S.pc[p] = S.ptot[p];
+      S.poff[p] = run;
+      run += S.pc[p];
     }
-    poff[E] = run;
+    S.poff[E] = run;
   }
   __syncthreads();
+  return R_exp;
+}
 
-  // 3. global counts and offsets (block 0)
-  if (b == 0) {
-    for (int e = tid; e < G; e += kLThreads) {
-      a.expert_count[e] = tot[e];
-      a.expert_offset[e] = eoff[e];
+__device__ void write_globals(const LayoutArgs& a, const Smem& S, int R_exp, int flags) {
+  for (int e = threadIdx.x; e < a.G; e += kLThreads) {
+    a.expert_count[e] = S.tot[e];
+    a.expert_offset[e] = S.eoff[e];
+  }
+  for (int p = threadIdx.x; p < a.E; p += kLThreads) {
+    a.part_count[p] = S.pc[p];
+    a.part_offset[p] = S.poff[p];
+  }
+  if (threadIdx.x == 0) {
+    a.expert_offset[a.G] = R_exp;
+    a.part_offset[a.E] = S.poff[a.E];
+    *a.status = flags;
+  }
+}
+
+// dedup: dispatch row of each distinct (token, partition) of the tile
+__device__ void rank_tile_parts(const LayoutArgs& a, const Tile& tl, const Smem& S,
+                                const RawIds& ids) {
+  const int E = a.E, lane = lane_id(), warp = warp_id(), tid = threadIdx.x;
+  const unsigned lt = lanemask_lt();
+  for (int r0 = 0; r0 < tl.ntok; r0 += kLThreads) {
+    const int t = r0 + tid;
+    const unsigned long long mask = t < tl.ntok ? token_mask(a, ids, S.part_s, t) : 0ull;
+    for (int p = 0; p < E; ++p) {
+      const unsigned bal = __ballot_sync(kFull, (mask >> p) & 1ull);
+      if (lane == 0) S.wp[warp * E + p] = __popc(bal);
     }
-    for (int p = tid; p < E; p += kLThreads) {
-      a.part_count[p] = pc[p];
-      a.part_offset[p] = poff[p];
-    }
-    int f = 0;
-    for (int r = tid; r < nt; r += kLThreads) f |= __ldcg(a.tile_flags + r);
-    if (f) atomicOr(&misc[0], f);
     __syncthreads();
-    if (tid == 0) {
-      a.expert_offset[G] = R_exp;
-      a.part_offset[E] = poff[E];
-      *a.status = misc[0];
+    for (int p = tid; p < E; p += kLThreads) {
+      int run = S.pbase[p];
+      for (int w = 0; w < kLWarps; ++w) {
+        const int v = S.wp[w * E + p];
+        S.wp[w * E + p] = run;
+        run += v;
+      }
+      S.pbase[p] = run;
     }
-  }
-
-  const int t0 = b * a.T;
-  const int ntok = max(0, min(a.M - t0, a.T));
-  const int n_items = ntok * a.topk;
-  const int* idx = a.idx + (size_t)t0 * a.topk;
-
-  // 4. dedup: dispatch row of each distinct (token, partition) of the tile
-  if (a.dedup) {
-    const unsigned lt = lanemask_lt();
-    for (int r0 = 0; r0 < ntok; r0 += kLThreads) {
-      const int tl = r0 + tid;
-      unsigned long long mask = 0ull;
-      if (tl < ntok) {
-        for (int k = 0; k < a.topk; ++k) {
-          const int e = __ldg(idx + (size_t)tl * a.topk + k);
-          if (e >= 0 && e < G) {
-            const int p = part_s[e];
-            if (valid_part(p, E)) mask |= 1ull << p;
-          }
+    __syncthreads();
+    const int tg = tl.t0 + t;
+    for (int p = 0; p < E; ++p) {
+      const bool has = (mask >> p) & 1ull;
+      const unsigned bal = __ballot_sync(kFull, has);
+      if (t < tl.ntok) {
+        int row = -1;
+        if (has) {
+          row = S.poff[p] + S.ppre[p] + S.wp[warp * E + p] + __popc(bal & lt);
+          a.disp_token[row] = tg;
         }
+        a.disp_row[(size_t)tg * E + p] = row;
       }
-      for (int p = 0; p < E; ++p) {
-        const unsigned bal = __ballot_sync(kFull, (mask >> p) & 1ull);
-        if (lane == 0) wp[warp * E + p] = __popc(bal);
-      }
-      __syncthreads();
-      for (int p = tid; p < E; p += kLThreads) {
-        int run = pbase[p];
-        for (int w = 0; w < kLWarps; ++w) {
-          const int v = wp[w * E + p];
-          wp[w * E + p] = run;
-          run += v;
-        }
-        pbase[p] = run;
-      }
-      __syncthreads();
-      const int t = t0 + tl;
-      for (int p = 0; p < E; ++p) {
-        const bool has = (mask >> p) & 1ull;
-        const unsigned bal = __ballot_sync(kFull, has);
-        if (tl < ntok) {
-          int row = -1;
-          if (has) {
-            row = poff[p] + ppre[p] + wp[warp * E + p] + __popc(bal & lt);
-            a.disp_token[row] = t;
-          }
-          a.disp_row[(size_t)t * E + p] = row;
-        }
-      }
-      __syncthreads();
     }
+    __syncthreads();
   }
+}
 
-  // 5. expert row of every pair of the tile, stable in (token, slot) order
-  for (int i = tid; i < kLWarps * G; i += kLThreads) whist[i] = 0;
-  __syncthreads();
+// expert row of every pair of the tile (second pass of the stable rank)
+__device__ void rank_tile_items(const LayoutArgs& a, const Tile& tl, const Smem& S,
+                                const RawIds& ids) {
+  const int G = a.G, E = a.E;
+  int* exp_row = a.exp_row + (size_t)tl.t0 * a.topk;
   auto ikey = [&](int i) {
-    const int e = __ldg(idx + i);
-    return (e >= 0 && e < G && valid_part(part_s[e], E)) ? e : -1;
+    const int e = ids(i);
+    return (e >= 0 && e < G && valid_part(S.part_s[e], E)) ? e : -1;
   };
-  int* exp_row = a.exp_row + (size_t)t0 * a.topk;
-  block_stable_rank(
-      n_items, G, whist, nullptr, ikey,
+  rank_assign(
+      tl.n_items, G, S.whist, ikey,
       [&](int i, int e, int r) {
-        const int row = eoff[e] + pre[e] + r;
+        const int row = S.eoff[e] + S.pre[e] + r;
         exp_row[i] = row;
-        const int t = t0 + i / a.topk;
+        const int t = tl.t0 + i / a.topk;
         if (!a.dedup) {
           a.disp_token[row] = t;
         } else {
-          a.exp_to_disp[row] = a.disp_row[(size_t)t * E + part_s[e]];
+          a.exp_to_disp[row] = a.disp_row[(size_t)t * E + S.part_s[e]];
         }
       },
       [&](int i) { exp_row[i] = -1; });
+}
+
+__device__ __forceinline__ int item_key(const LayoutArgs& a, const Smem& S, const RawIds& ids,
+                                        int i) {
+  const int e = ids(i);
+  return (e >= 0 && e < a.G && valid_part(S.part_s[e], a.E)) ? e : -1;
+}
+
+// ---------------------------------------------------------------------------
+// schedule 1: one cluster
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kLThreads) layout_cluster_kernel(LayoutArgs a) {
+  extern __shared__ __align__(16) int sm[];
+  cg::cluster_group cluster = cg::this_cluster();
+  const LayoutSmem P(a.G, a.E, a.key_cap);
+  const Smem S(sm, P);
+  const int r = (int)cluster.block_rank();
+  const int tid = threadIdx.x;
+  const Tile tl = tile_of(a, r);
+  RawIds ids;
+  stage_tile(a, tl, S, ids);
+
+  // count the tile; the per-warp bases stay in whist for the ranks below
+  const int f = scan_flags(a, tl, S, ids, r == 0);
+  if (f) atomicOr(&S.misc[0], f);
+  rank_count(tl.n_items, a.G, S.whist, S.cta_hist, [&](int i) { return item_key(a, S, ids, i); });
+  if (a.dedup) count_tile_parts(a, tl, S, ids);
+  cluster.sync();
+
+  // exchange: totals over the cluster and the prefix of the tiles before r
+  for (int e = tid; e < a.G; e += kLThreads) {
+    int v[kClusterCTAs];
+#pragma unroll
+    for (int q = 0; q < kClusterCTAs; ++q) v[q] = cluster.map_shared_rank(S.cta_hist, q)[e];
+    int all = 0, bef = 0;
+#pragma unroll
+    for (int q = 0; q < kClusterCTAs; ++q) {
+      all += v[q];
+      bef += q < r ? v[q] : 0;
+    }
+    S.tot[e] = all;
+    S.pre[e] = bef;
+  }
+  if (a.dedup) {
+    for (int p = tid; p < a.E; p += kLThreads) {
+      int all = 0, bef = 0;
+      for (int q = 0; q < kClusterCTAs; ++q) {
+        const int v = cluster.map_shared_rank(S.cta_phist, q)[p];
+        all += v;
+        bef += q < r ? v : 0;
+      }
+      S.ptot[p] = all;
+      S.ppre[p] = bef;
+    }
+  }
+  int flags = 0;
+  if (r == 0 && tid < kClusterCTAs) flags = cluster.map_shared_rank(S.misc, tid)[0];
+  __syncthreads();
+  if (r == 0 && flags) atomicOr(&S.misc[1], flags);
+
+  const int R_exp = finish_offsets(a, S);
+  if (r == 0) write_globals(a, S, R_exp, S.misc[1]);
+  if (a.dedup) rank_tile_parts(a, tl, S, ids);
+  rank_tile_items(a, tl, S, ids);
+  cluster.sync();  // no block leaves while another may still read its histograms
+}
+
+// ---------------------------------------------------------------------------
+// schedule 2: one tile per SM, two launches
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kLThreads) layout_count_kernel(LayoutArgs a) {
+  extern __shared__ __align__(16) int sm[];
+  const LayoutSmem P(a.G, a.E, a.key_cap);
+  const Smem S(sm, P);
+  const int b = blockIdx.x;
+  const Tile tl = tile_of(a, b);
+  RawIds ids;
+  stage_tile(a, tl, S, ids);
+  const int f = scan_flags(a, tl, S, ids, b == 0);
+  if (f) atomicOr(&S.misc[0], f);
+  rank_count(tl.n_items, a.G, S.whist, S.cta_hist, [&](int i) { return item_key(a, S, ids, i); });
+  if (a.dedup) count_tile_parts(a, tl, S, ids);
+  int* th = a.tile_hist + (size_t)b * a.G;
+  for (int i = threadIdx.x; i < a.G; i += kLThreads) th[i] = S.cta_hist[i];
+  if (a.dedup)
+    for (int i = threadIdx.x; i < a.E; i += kLThreads)
+      a.tile_phist[(size_t)b * a.E + i] = S.cta_phist[i];
+  if (threadIdx.x == 0) a.tile_flags[b] = S.misc[0];
+}
+
+// Column sums of a [rows][cols] int matrix in global memory (L2): total over
+// all rows and over rows < b.  Each thread keeps up to 8 16-byte loads in
+// flight.  `red` holds 2 * kRedW ints (cols <= MOE_MAX_G <= kRedW).
+__device__ void column_sums(const int* src, int rows, int cols, int b, int* red, int* total,
+                            int* before) {
+  const int tid = threadIdx.x;
+  const int RW = kRedW;
+  const bool vec = (cols & 3) == 0 && (reinterpret_cast<uintptr_t>(src) & 15) == 0;
+  if (vec) {
+    const int C4 = cols >> 2;
+    const int S = C4 <= kLThreads ? kLThreads / C4 : 1;
+    for (int slot = tid; slot < C4 * S; slot += kLThreads) {
+      const int c4 = slot % C4, s = slot / C4;
+      int4 all = make_int4(0, 0, 0, 0), bef = all;
+#pragma unroll 8
+      for (int r = s; r < rows; r += S) {
+        const int4 v = __ldcg(reinterpret_cast<const int4*>(src + (size_t)r * cols) + c4);
+        all.x += v.x; all.y += v.y; all.z += v.z; all.w += v.w;
+        if (r < b) {
+          bef.x += v.x; bef.y += v.y; bef.z += v.z; bef.w += v.w;
+        }
+      }
+      const int base = s * cols + 4 * c4;
+      red[base] = all.x; red[base + 1] = all.y; red[base + 2] = all.z; red[base + 3] = all.w;
+      red[RW + base] = bef.x; red[RW + base + 1] = bef.y;
+      red[RW + base + 2] = bef.z; red[RW + base + 3] = bef.w;
+    }
+    __syncthreads();
+    for (int c = tid; c < cols; c += kLThreads) {
+      int all = 0, bef = 0;
+      for (int s = 0; s < S; ++s) {
+        all += red[s * cols + c];
+        bef += red[RW + s * cols + c];
+      }
+      total[c] = all;
+      before[c] = bef;
+    }
+  } else {
+    const int S = cols <= kLThreads ? kLThreads / cols : 1;
+    for (int slot = tid; slot < cols * S; slot += kLThreads) {
+      const int c = slot % cols, s = slot / cols;
+      int all = 0, bef = 0;
+#pragma unroll 8
+      for (int r = s; r < rows; r += S) {
+        const int v = __ldcg(src + (size_t)r * cols + c);
+        all += v;
+        bef += (r < b) ? v : 0;
+      }
+      red[slot] = all;
+      red[RW + slot] = bef;
+    }
+    __syncthreads();
+    for (int c = tid; c < cols; c += kLThreads) {
+      int all = 0, bef = 0;
+      for (int s = 0; s < S; ++s) {
+        all += red[s * cols + c];
+        bef += red[RW + s * cols + c];
+      }
+      total[c] = all;
+      before[c] = bef;
+    }
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kLThreads) layout_rank_kernel(LayoutArgs a) {
+  extern __shared__ __align__(16) int sm[];
+  const LayoutSmem P(a.G, a.E, a.key_cap);
+  const Smem S(sm, P);
+  const int b = blockIdx.x;
+  const Tile tl = tile_of(a, b);
+  RawIds ids;
+  stage_tile(a, tl, S, ids);
+
+  column_sums(a.tile_hist, a.n_tiles, a.G, b, S.red, S.tot, S.pre);
+  if (a.dedup) column_sums(a.tile_phist, a.n_tiles, a.E, b, S.red, S.ptot, S.ppre);
+  rank_count(tl.n_items, a.G, S.whist, nullptr, [&](int i) { return item_key(a, S, ids, i); });
+
+  const int R_exp = finish_offsets(a, S);
+  if (b == 0) {
+    int f = 0;
+    for (int q = threadIdx.x; q < a.n_tiles; q += kLThreads) f |= __ldcg(a.tile_flags + q);
+    if (f) atomicOr(&S.misc[1], f);
+    __syncthreads();
+    write_globals(a, S, R_exp, S.misc[1]);
+  }
+  if (a.dedup) rank_tile_parts(a, tl, S, ids);
+  rank_tile_items(a, tl, S, ids);
+}
+
+bool use_cluster(const moe_problem_t& p) { return (int64_t)p.M * p.topk <= kClusterItems; }
+
+size_t smem_bytes(const moe_problem_t& p, int key_cap) {
+  return sizeof(int) * (size_t)LayoutSmem(p.G, p.E_part, key_cap).total;
 }
 
 }  // namespace
@@ -458,7 +637,7 @@ __global__ void __launch_bounds__(kLThreads) layout_rank_kernel(LayoutArgs a) {
 int layout_tile_tokens(int M) {
   int t = (M + 147) / 148;
   t = (t + 31) / 32 * 32;
-  return std::max(64, t);
+  return std::max(MOE_TILE_MIN_TOKENS, t);
 }
 
 int layout_num_tiles(int M) {
@@ -481,14 +660,8 @@ cudaError_t launch_layout(const moe_problem_t& p, const int32_t* topk_idx,
   a.topk = p.topk;
   a.E = p.E_part;
   a.dedup = p.dedup;
-  a.T = layout_tile_tokens(p.M);
-  a.n_tiles = layout_num_tiles(p.M);
   a.idx = topk_idx;
   a.part_of = part_of;
-  int* ws = static_cast<int*>(workspace);
-  a.tile_hist = ws;
-  a.tile_phist = ws + (size_t)a.n_tiles * p.G;
-  a.tile_flags = a.tile_phist + (p.dedup ? (size_t)a.n_tiles * p.E_part : 0);
   a.expert_count = lay.expert_count;
   a.expert_offset = lay.expert_offset;
   a.part_count = lay.part_count;
@@ -499,17 +672,48 @@ cudaError_t launch_layout(const moe_problem_t& p, const int32_t* topk_idx,
   a.exp_to_disp = lay.exp_to_disp;
   a.status = lay.status;
 
-  const size_t smem1 = sizeof(int) * (2 * (size_t)p.G + p.E_part);
-  const size_t smem2 = sizeof(int) * (size_t)RankSmem(p.G, p.E_part).total;
-  if (smem2 > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(layout_rank_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2);
+  if (use_cluster(p)) {
+    // tiles of a multiple of 4 tokens keep every tile's ids 16-byte aligned
+    a.T = std::max(4, ((p.M + kClusterCTAs - 1) / kClusterCTAs + 3) / 4 * 4);
+    a.n_tiles = kClusterCTAs;
+    a.key_cap = a.T * p.topk;
+    a.tile_hist = a.tile_phist = a.tile_flags = nullptr;
+    const size_t smem = smem_bytes(p, a.key_cap);
+    cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void*>(layout_cluster_kernel), smem);
     if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kClusterCTAs);
+    cfg.blockDim = dim3(kLThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kClusterCTAs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, layout_cluster_kernel, a);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
   }
-  layout_count_kernel<<<a.n_tiles, kLThreads, smem1, stream>>>(a);
-  cudaError_t e = cudaGetLastError();
+
+  a.T = layout_tile_tokens(p.M);
+  a.n_tiles = layout_num_tiles(p.M);
+  a.key_cap = a.T * p.topk <= kMaxTileItems ? a.T * p.topk : 0;
+  int* ws = static_cast<int*>(workspace);
+  a.tile_hist = ws;
+  a.tile_phist = ws + (size_t)a.n_tiles * p.G;
+  a.tile_flags = a.tile_phist + (p.dedup ? (size_t)a.n_tiles * p.E_part : 0);
+  const size_t smem = smem_bytes(p, a.key_cap);
+  cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void*>(layout_count_kernel), smem);
   if (e != cudaSuccess) return e;
-  layout_rank_kernel<<<a.n_tiles, kLThreads, smem2, stream>>>(a);
+  e = allow_dynamic_smem(reinterpret_cast<const void*>(layout_rank_kernel), smem);
+  if (e != cudaSuccess) return e;
+  layout_count_kernel<<<a.n_tiles, kLThreads, smem, stream>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  layout_rank_kernel<<<a.n_tiles, kLThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }
 

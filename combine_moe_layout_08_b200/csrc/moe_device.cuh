@@ -52,6 +52,55 @@ __device__ __forceinline__ void st_cs_v4(void* p, const uint4& v) {
                : "memory");
 }
 
+// W 32-bit words moved as one vector: W = 4 (16 bytes) or W = 8 (32 bytes,
+// 256-bit loads and stores on sm_100a; addresses 32-byte aligned).
+template <int W>
+struct Vec {
+  uint32_t w[W];
+};
+
+template <int W>
+__device__ __forceinline__ Vec<W> ld_nc(const void* p);
+
+template <>
+__device__ __forceinline__ Vec<4> ld_nc<4>(const void* p) {
+  Vec<4> v;
+  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+      : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3])
+      : "l"(p));
+  return v;
+}
+
+template <>
+__device__ __forceinline__ Vec<8> ld_nc<8>(const void* p) {
+  Vec<8> v;
+  asm("ld.global.nc.L1::no_allocate.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+      : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3]), "=r"(v.w[4]), "=r"(v.w[5]),
+        "=r"(v.w[6]), "=r"(v.w[7])
+      : "l"(p));
+  return v;
+}
+
+template <int W>
+__device__ __forceinline__ void st_na(void* p, const Vec<W>& v);
+
+template <>
+__device__ __forceinline__ void st_na<4>(void* p, const Vec<4>& v) {
+  asm volatile("st.global.L1::no_allocate.v4.u32 [%0], {%1, %2, %3, %4};"
+               :
+               : "l"(p), "r"(v.w[0]), "r"(v.w[1]), "r"(v.w[2]), "r"(v.w[3])
+               : "memory");
+}
+
+template <>
+__device__ __forceinline__ void st_na<8>(void* p, const Vec<8>& v) {
+  asm volatile("st.global.L1::no_allocate.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+               :
+               : "l"(p), "r"(v.w[0]), "r"(v.w[1]), "r"(v.w[2]), "r"(v.w[3]), "r"(v.w[4]),
+                 "r"(v.w[5]), "r"(v.w[6]), "r"(v.w[7])
+               : "memory");
+}
+
 __device__ __forceinline__ int ld_nc_i32(const int* p) {
   int v;
   asm("ld.global.nc.L1::no_allocate.b32 %0, [%1];" : "=r"(v) : "l"(p));
@@ -68,6 +117,24 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 }
 
 __device__ __forceinline__ int lane_id() { return threadIdx.x & (kWarp - 1); }
+
+// Lanes of the warp holding the same key as this lane (all lanes active).
+// Keys are in [-1, 2^nbits - 1): -1 (all ones in the low nbits bits) is a key
+// of its own.  One ballot per key bit, intersected: on sm_100a this runs at
+// the vote rate on every sub-partition, several times the throughput of
+// match.any.
+__device__ __forceinline__ unsigned match_peers(int key, int nbits) {
+  unsigned m = kFull;
+  for (int b = 0; b < nbits; ++b) {
+    const bool bit = (key >> b) & 1;
+    const unsigned bal = __ballot_sync(kFull, bit);
+    m &= bit ? bal : ~bal;
+  }
+  return m;
+}
+
+// Key bits for keys in [-1, K): enough that K - 1 < 2^nbits - 1.
+__device__ __forceinline__ int key_bits(int K) { return 32 - __clz(K); }
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
 
 // ---------------------------------------------------------------------------

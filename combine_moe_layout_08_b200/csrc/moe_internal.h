@@ -10,6 +10,16 @@
 
 namespace moe {
 
+// Resident blocks of `kernel` at `threads` per block and `smem` bytes of
+// dynamic shared memory on the whole current device (SM count x blocks per
+// SM), looked up once per device and configuration.  Grids of persistent
+// kernels are sized with it.
+int device_block_slots(const void* kernel, int threads, size_t smem = 0);
+
+// Raise `kernel`'s dynamic shared-memory limit on the current device to at
+// least `bytes` (once per device and kernel; no-op up to 48 KB).
+cudaError_t allow_dynamic_smem(const void* kernel, size_t bytes);
+
 // Tokens per layout tile: about one tile per SM, at least 64 tokens, a
 // multiple of 32.
 int layout_tile_tokens(int M);

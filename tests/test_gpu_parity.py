@@ -103,6 +103,10 @@ SHAPES = [
     (70001, 8, 256, 8, 8, True, False, "uniform"),   # many tiles, layout-heavy
     (4097, 384, 48, 6, 5, False, True, "zipf"),
     (2048, 7168, 256, 8, 8, True, True, "uniform"),
+    (1024, 64, 256, 8, 8, True, False, "zipf"),      # 8192 pairs: largest one-cluster layout
+    (1025, 64, 256, 8, 8, True, False, "zipf"),      # 8200 pairs: two-launch layout
+    (16385, 64, 256, 8, 8, True, False, "zipf"),
+    (310001, 8, 256, 8, 8, True, False, "uniform"),  # tiles too big for the id cache
 ]
 
 
@@ -259,3 +263,32 @@ def test_streams_and_graph_capture():
     ref = oracle.layout(idx, po, w.G, w.E_part, False)
     compare_combine(b, prob, y, gates, ref["exp_row"])
     del g
+
+
+@pytest.mark.parametrize("fp8,dedup", [(False, False), (True, True)])
+def test_buffers_only_16_byte_aligned(fp8, dedup):
+    """Rows that allow 32-byte vectors but buffers that start 16 bytes past a
+    32-byte boundary take the 16-byte paths; results are the same."""
+    w = _custom(777, 1024, 64, 6, 8, dedup=dedup, fp8=fp8, seed=9)
+    idx, po, gates, x0, y0 = _inputs(w)
+    prob = problem_of(w)
+
+    def shifted(t):
+        off = 16 // t.element_size()               # 16 bytes, whatever the dtype
+        flat = torch.empty(t.numel() + off, dtype=t.dtype, device=t.device)
+        v = flat[off:].view(t.shape)
+        v.copy_(t)
+        assert v.data_ptr() % 32 == 16
+        return v
+
+    x, y = shifted(x0), shifted(y0)
+    b = moe.MoEBuffers(prob, DEV)
+    b.recv_x = shifted(b.recv_x.view(torch.uint8 if fp8 else torch.bfloat16))
+    b.out = shifted(b.out)
+    b.layout_(to_dev(idx), to_dev(po))
+    b.dispatch_(x)
+    b.combine_(y, to_dev(gates))
+    torch.cuda.synchronize()
+    ref = oracle.layout(idx, po, w.G, w.E_part, w.dedup)
+    compare_dispatch_rows(b, prob, oracle.bf16_bits(x0), ref["disp_token"])
+    assert compare_combine(b, prob, y0, gates, ref["exp_row"]) == 0
