@@ -47,6 +47,8 @@ __global__ void __launch_bounds__(kCThreads) combine_kernel(CombineArgs a) {
   __shared__ float wts[MOE_MAX_TOPK];
   const int t = blockIdx.x;
   const int tid = threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
   if (tid < a.topk) {
     const int r = ld_nc_i32(a.exp_row + (size_t)t * a.topk + tid);
     const bool ok = r >= 0 && r < a.cap;
@@ -103,7 +105,8 @@ __global__ void __launch_bounds__(kCThreads) combine_kernel(CombineArgs a) {
 template <int KG, int U>
 cudaError_t launch(const CombineArgs& a, int M, cudaStream_t stream) {
   const dim3 grid(M, (a.N8 + kCThreads * U - 1) / (kCThreads * U));
-  combine_kernel<KG, U><<<grid, kCThreads, 0, stream>>>(a);
+  const cudaError_t e = launch_pdl(combine_kernel<KG, U>, grid, dim3(kCThreads), 0, stream, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -32,12 +32,34 @@ struct DispatchArgs {
   int N8;                       // 16-byte chunks per bf16 row (N / 8)
   int topk, E, dedup;
   int cap;                      // receive capacity in rows (M * topk)
+  int M;
+  int prefetch_stride;          // blocks [0, stride) warm L2 with rows b, b + stride, ...
+  int prefetch_rows;            // ... below this row (the first rows processed)
   const int* exp_row;           // [M][topk]
   const int* disp_row;          // [M][E], dedup only
   void* recv;                   // [cap][N] bf16 or u8
   float* recv_scale;            // [cap][N / 128], fp8 only
   int* status;
 };
+
+// While the previous kernel (the routing layout) still runs, the blocks that
+// are already resident warm L2 with the first token rows: block b < stride
+// prefetches rows b, b + stride, ... (stride = resident blocks) up to
+// kPrefetchBytes in all -- a third of L2, so the prefetched rows are still
+// there when their blocks run -- and those rows come from L2 once the
+// destinations are known.
+#ifndef MOE_DISPATCH_PREFETCH
+#define MOE_DISPATCH_PREFETCH 1
+#endif
+constexpr size_t kPrefetchBytes = 40u << 20;
+
+__device__ __forceinline__ void prefetch_rows(const DispatchArgs& a) {
+  if (!MOE_DISPATCH_PREFETCH) return;
+  if (threadIdx.x != 0 || blockIdx.y != 0 || (int)blockIdx.x >= a.prefetch_stride) return;
+  const uint32_t row_bytes = (uint32_t)a.N8 * 16u;
+  for (int t = blockIdx.x; t < a.prefetch_rows; t += a.prefetch_stride)
+    prefetch_l2(a.x + (size_t)t * a.N8, row_bytes);
+}
 
 // Destination rows of token t, in slot (or partition) order, into smem.
 __device__ __forceinline__ int destinations(const DispatchArgs& a, int t, int* dst, int* nd) {
@@ -64,12 +86,15 @@ __device__ __forceinline__ int destinations(const DispatchArgs& a, int t, int* d
 }
 
 template <int U>
-__global__ void __launch_bounds__(kDThreads) dispatch_bf16_kernel(DispatchArgs a) {
+__global__ void __launch_bounds__(kDThreads, 8) dispatch_bf16_kernel(DispatchArgs a) {
   __shared__ int dst[kMaxDest];
   __shared__ int nd;
   const int t = blockIdx.x;
   const int c0 = blockIdx.y * (kDThreads * U) + threadIdx.x;
   const uint4* src = a.x + (size_t)t * a.N8;
+  prefetch_rows(a);
+  pdl_wait();
+  pdl_trigger();
   uint4 v[U];
 #pragma unroll
   for (int u = 0; u < U; ++u) {
@@ -120,13 +145,16 @@ __device__ __forceinline__ float absmax8(const uint4& v) {
 // 128-column scale block.  N is a multiple of 128 and kDThreads of 8, so a
 // lane group is either entirely inside the row or entirely past its end.
 template <int U>
-__global__ void __launch_bounds__(kDThreads) dispatch_fp8_kernel(DispatchArgs a) {
+__global__ void __launch_bounds__(kDThreads, 8) dispatch_fp8_kernel(DispatchArgs a) {
   __shared__ int dst[kMaxDest];
   __shared__ int nd;
   const int t = blockIdx.x;
   const int N16 = a.N8 >> 1;
   const int g0 = blockIdx.y * (kDThreads * U) + threadIdx.x;
   const uint4* src = a.x + (size_t)t * a.N8;
+  prefetch_rows(a);
+  pdl_wait();
+  pdl_trigger();
   uint4 lo[U], hi[U];
 #pragma unroll
   for (int u = 0; u < U; ++u) {
@@ -186,6 +214,7 @@ cudaError_t launch_dispatch(const moe_problem_t& p, const void* x, const moe_lay
   a.E = p.E_part;
   a.dedup = p.dedup;
   a.cap = p.M * p.topk;
+  a.M = p.M;
   a.exp_row = lay.exp_row;
   a.disp_row = lay.disp_row;
   a.recv = recv_x;
@@ -198,25 +227,36 @@ cudaError_t launch_dispatch(const moe_problem_t& p, const void* x, const moe_lay
   const int U = std::min(Umax, (units + kDThreads - 1) / kDThreads);
   const int per_block = kDThreads * U;
   dim3 grid(p.M, (units + per_block - 1) / per_block);
+  // blocks resident at once on this device (an estimate from the register
+  // budget of the widest variant; only the L2 prefetch uses it)
+  a.prefetch_stride = std::max(1, std::min(p.M, device_block_slots(
+      reinterpret_cast<const void*>(dispatch_bf16_kernel<8>), kDThreads) / (int)grid.y));
+  // measured on B200: the prefetch pays when every row fans out to many
+  // copies (HBM busy writing); with dedup or small topk it only adds L2
+  // pressure
+  const bool fan_out = !p.dedup && p.topk >= 4;
+  a.prefetch_rows = fan_out ? (int)std::min<size_t>((size_t)p.M, kPrefetchBytes / (2 * (size_t)p.N)) : 0;
+  cudaError_t e = cudaSuccess;
   if (!p.fp8) {
     switch (U) {
-      case 1: dispatch_bf16_kernel<1><<<grid, kDThreads, 0, stream>>>(a); break;
-      case 2: dispatch_bf16_kernel<2><<<grid, kDThreads, 0, stream>>>(a); break;
-      case 3: dispatch_bf16_kernel<3><<<grid, kDThreads, 0, stream>>>(a); break;
-      case 4: dispatch_bf16_kernel<4><<<grid, kDThreads, 0, stream>>>(a); break;
-      case 5: dispatch_bf16_kernel<5><<<grid, kDThreads, 0, stream>>>(a); break;
-      case 6: dispatch_bf16_kernel<6><<<grid, kDThreads, 0, stream>>>(a); break;
-      case 7: dispatch_bf16_kernel<7><<<grid, kDThreads, 0, stream>>>(a); break;
-      default: dispatch_bf16_kernel<8><<<grid, kDThreads, 0, stream>>>(a); break;
+      case 1: e = launch_pdl(dispatch_bf16_kernel<1>, grid, dim3(kDThreads), 0, stream, a); break;
+      case 2: e = launch_pdl(dispatch_bf16_kernel<2>, grid, dim3(kDThreads), 0, stream, a); break;
+      case 3: e = launch_pdl(dispatch_bf16_kernel<3>, grid, dim3(kDThreads), 0, stream, a); break;
+      case 4: e = launch_pdl(dispatch_bf16_kernel<4>, grid, dim3(kDThreads), 0, stream, a); break;
+      case 5: e = launch_pdl(dispatch_bf16_kernel<5>, grid, dim3(kDThreads), 0, stream, a); break;
+      case 6: e = launch_pdl(dispatch_bf16_kernel<6>, grid, dim3(kDThreads), 0, stream, a); break;
+      case 7: e = launch_pdl(dispatch_bf16_kernel<7>, grid, dim3(kDThreads), 0, stream, a); break;
+      default: e = launch_pdl(dispatch_bf16_kernel<8>, grid, dim3(kDThreads), 0, stream, a); break;
     }
   } else {
     switch (U) {
-      case 1: dispatch_fp8_kernel<1><<<grid, kDThreads, 0, stream>>>(a); break;
-      case 2: dispatch_fp8_kernel<2><<<grid, kDThreads, 0, stream>>>(a); break;
-      case 3: dispatch_fp8_kernel<3><<<grid, kDThreads, 0, stream>>>(a); break;
-      default: dispatch_fp8_kernel<4><<<grid, kDThreads, 0, stream>>>(a); break;
+      case 1: e = launch_pdl(dispatch_fp8_kernel<1>, grid, dim3(kDThreads), 0, stream, a); break;
+      case 2: e = launch_pdl(dispatch_fp8_kernel<2>, grid, dim3(kDThreads), 0, stream, a); break;
+      case 3: e = launch_pdl(dispatch_fp8_kernel<3>, grid, dim3(kDThreads), 0, stream, a); break;
+      default: e = launch_pdl(dispatch_fp8_kernel<4>, grid, dim3(kDThreads), 0, stream, a); break;
     }
   }
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -465,6 +465,8 @@ __global__ void __launch_bounds__(kLThreads) layout_cluster_kernel(LayoutArgs a)
   const int r = (int)cluster.block_rank();
   const int tid = threadIdx.x;
   const Tile tl = tile_of(a, r);
+  pdl_wait();
+  pdl_trigger();
   RawIds ids;
   stage_tile(a, tl, S, ids);
 
@@ -522,6 +524,8 @@ __global__ void __launch_bounds__(kLThreads) layout_count_kernel(LayoutArgs a) {
   const Smem S(sm, P);
   const int b = blockIdx.x;
   const Tile tl = tile_of(a, b);
+  pdl_wait();
+  pdl_trigger();
   RawIds ids;
   stage_tile(a, tl, S, ids);
   const int f = scan_flags(a, tl, S, ids, b == 0);
@@ -607,8 +611,12 @@ __global__ void __launch_bounds__(kLThreads) layout_rank_kernel(LayoutArgs a) {
   const Smem S(sm, P);
   const int b = blockIdx.x;
   const Tile tl = tile_of(a, b);
+  // the caller's inputs were complete before layout_count_kernel started,
+  // so they are staged before waiting for its histograms
   RawIds ids;
   stage_tile(a, tl, S, ids);
+  pdl_wait();
+  pdl_trigger();
 
   column_sums(a.tile_hist, a.n_tiles, a.G, b, S.red, S.tot, S.pre);
   if (a.dedup) column_sums(a.tile_phist, a.n_tiles, a.E, b, S.red, S.ptot, S.ppre);
@@ -686,13 +694,15 @@ cudaError_t launch_layout(const moe_problem_t& p, const int32_t* topk_idx,
     cfg.blockDim = dim3(kLThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = kClusterCTAs;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = MOE_USE_PDL;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     e = cudaLaunchKernelEx(&cfg, layout_cluster_kernel, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
@@ -710,10 +720,10 @@ cudaError_t launch_layout(const moe_problem_t& p, const int32_t* topk_idx,
   if (e != cudaSuccess) return e;
   e = allow_dynamic_smem(reinterpret_cast<const void*>(layout_rank_kernel), smem);
   if (e != cudaSuccess) return e;
-  layout_count_kernel<<<a.n_tiles, kLThreads, smem, stream>>>(a);
-  e = cudaGetLastError();
+  e = launch_pdl(layout_count_kernel, dim3(a.n_tiles), dim3(kLThreads), smem, stream, a);
   if (e != cudaSuccess) return e;
-  layout_rank_kernel<<<a.n_tiles, kLThreads, smem, stream>>>(a);
+  e = launch_pdl(layout_rank_kernel, dim3(a.n_tiles), dim3(kLThreads), smem, stream, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

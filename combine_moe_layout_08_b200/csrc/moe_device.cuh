@@ -101,6 +101,14 @@ __device__ __forceinline__ void st_na<8>(void* p, const Vec<8>& v) {
                : "memory");
 }
 
+// Bulk prefetch of [p, p + bytes) into L2 (no registers, no shared memory;
+// 16-byte aligned, bytes a multiple of 16).  Always safe to issue early: L2
+// is the GPU's point of coherence, so a line prefetched before its last
+// writer finishes is simply updated in place.
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ int ld_nc_i32(const int* p) {
   int v;
   asm("ld.global.nc.L1::no_allocate.b32 %0, [%1];" : "=r"(v) : "l"(p));
@@ -148,6 +156,19 @@ __device__ __forceinline__ uint32_t pack_bf16x2_rn(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// ---------------------------------------------------------------------------
+// programmatic dependent launch (sm_90+).  A kernel launched with the
+// programmatic-serialisation attribute may start while the previous kernel
+// in the stream is still running; pdl_wait() blocks (in hardware) until that
+// kernel has completed and its memory is visible, and pdl_trigger() lets the
+// next such kernel start once every block of this one has passed it.  In a
+// kernel launched without the attribute both are no-ops.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------

@@ -6,7 +6,13 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include <utility>
+
 #include "moe_layout.h"
+
+#ifndef MOE_USE_PDL
+#define MOE_USE_PDL 1  // programmatic dependent launch between the path's kernels
+#endif
 
 namespace moe {
 
@@ -15,6 +21,25 @@ namespace moe {
 // SM), looked up once per device and configuration.  Grids of persistent
 // kernels are sized with it.
 int device_block_slots(const void* kernel, int threads, size_t smem = 0);
+
+// Launch `kernel` with programmatic stream serialisation (it may start while
+// the previous kernel in `stream` runs; it must pdl_wait() before reading
+// anything that kernel writes).
+template <class... KArgs, class... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = MOE_USE_PDL;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Raise `kernel`'s dynamic shared-memory limit on the current device to at
 // least `bytes` (once per device and kernel; no-op up to 48 KB).
