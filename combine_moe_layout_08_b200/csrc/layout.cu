@@ -12,19 +12,27 @@
 // of expert e start at  expert_offset[e] + (rows of e in earlier tiles), and
 // inside the tile they are ranked stably in (token, slot) order: each warp
 // counts its contiguous segment into a warp-private histogram, an exclusive
-// scan across warps gives each warp's base, and a ballot match (one vote per key
-// bit) ranks the lanes of a 32-pair chunk.  Everything is fixed by the data, so the result is
-// bitwise reproducible.
+// scan across warps gives each warp's base, and a ballot match (one vote per
+// key bit) ranks the lanes of a 32-pair chunk.  Everything is fixed by the
+// data, so the result is bitwise reproducible.
+//
+// Each tile summarises itself in one row of W ints: its count per expert,
+// with dedup its distinct (token, partition) count per partition, and two
+// counters of invalid input (expert ids outside [0, G); placement entries
+// outside [0, E_part), first tile only).  One column reduction over the rows
+// then gives every total, every tile prefix and the status word.
 //
 // Two schedules, no host round trip in either:
-//   * up to kClusterItems routed pairs (decode-sized batches): ONE launch of
-//     a cluster of kClusterCTAs blocks.  Each block counts its tile into shared memory,
-//     the blocks exchange their tile histograms through distributed shared
-//     memory between two hardware cluster barriers, and every block finishes
-//     its own tile.  No workspace is touched.
-//   * larger batches: one tile per SM in two launches -- layout_count_kernel
-//     writes per-tile histograms to the workspace, layout_rank_kernel reduces
-//     them (batched 16-byte loads from L2) and ranks its tile.
+//   * small batches (<= kClusterItems routed pairs): ONE launch of a cluster
+//     of C <= 8 blocks (one per MOE_CLUSTER_BLOCK_ITEMS pairs); the blocks
+//     exchange their rows through distributed shared memory between two
+//     hardware cluster barriers.  No workspace is touched.
+//   * larger batches: about one tile per SM in two launches.
+//     layout_count_kernel writes the rows to the workspace;
+//     layout_rank_kernel stages its tile, counts it per warp and orders the
+//     experts by (partition, id) -- all from the caller's inputs, before it
+//     waits for layout_count_kernel (programmatic dependent launch) -- then
+//     reduces the rows with batched 16-byte loads from L2 and ranks its tile.
 // In both, the tile's expert ids are cached in shared memory when they fit.
 #include <cooperative_groups.h>
 
@@ -40,34 +48,45 @@ namespace {
 
 constexpr int kLThreads = 512;
 constexpr int kLWarps = kLThreads / kWarp;
-constexpr int kClusterCTAs = 8;
+constexpr int kMaxCluster = 8;
 constexpr int kMaxTileItems = 16384;  // tile ids cached in shared memory (64 KB)
 // Compile-time tuning constants: batches of at most MOE_CLUSTER_ITEMS routed
-// pairs take the one-cluster schedule; tiles of the two-launch schedule hold
-// at least MOE_TILE_MIN_TOKENS tokens.
+// pairs take the one-cluster schedule, with one block per
+// MOE_CLUSTER_BLOCK_ITEMS pairs; tiles of the two-launch schedule hold at
+// least MOE_TILE_MIN_TOKENS tokens.
 #ifndef MOE_CLUSTER_ITEMS
 #define MOE_CLUSTER_ITEMS 8192  // measured on B200: one cluster wins only for small batches
 #endif
+#ifndef MOE_CLUSTER_BLOCK_ITEMS
+#define MOE_CLUSTER_BLOCK_ITEMS 256  // measured on B200 (decode batch: 4 blocks beat 1)
+#endif
 #ifndef MOE_TILE_MIN_TOKENS
-#define MOE_TILE_MIN_TOKENS 64
+#define MOE_TILE_MIN_TOKENS 128  // measured on B200 (64..256 within noise; 128 best for fp8)
 #endif
 constexpr int kClusterItems = MOE_CLUSTER_ITEMS;
-static_assert(kClusterItems <= kClusterCTAs * kMaxTileItems, "cluster tiles must fit the id cache");
-// width of each half of the column-sum reduction buffer: one slot per thread
-// and 4 columns per slot (>= MOE_MAX_G, the widest matrix reduced)
+static_assert(kClusterItems <= kMaxCluster * kMaxTileItems, "cluster tiles must fit the id cache");
+// width of each half of the column-sum reduction buffer: one slot per thread,
+// 4 columns per slot, and at least the widest tile row (MOE_MAX_G +
+// MOE_MAX_E_PART + 2, padded)
 constexpr int kRedW = 4 * kLThreads;
-static_assert(kRedW >= MOE_MAX_G, "reduction buffer narrower than the expert count");
+static_assert(kRedW >= MOE_MAX_G + MOE_MAX_E_PART + 4, "reduction buffer narrower than a tile row");
+
+__host__ __device__ constexpr int up4(int x) { return (x + 3) & ~3; }
+
+// ints per tile row: [G expert counts | E partition counts (dedup) | 2 flag counts], padded
+__host__ __device__ constexpr int row_width(int G, int E, int dedup) {
+  return up4(G + (dedup ? E : 0) + 2);
+}
 
 struct LayoutArgs {
   int M, G, topk, E, dedup;
   int T;        // tokens per tile
   int n_tiles;  // tiles (= blocks)
   int key_cap;  // ids the shared-memory cache holds (0: read from global)
+  int W;        // ints per tile row
   const int* __restrict__ idx;
   const int* __restrict__ part_of;
-  int* tile_hist;   // [n_tiles][G]   (two-launch schedule)
-  int* tile_phist;  // [n_tiles][E]   (two-launch schedule, dedup)
-  int* tile_flags;  // [n_tiles]      (two-launch schedule)
+  int* tile_rows;  // [n_tiles][W]   (two-launch schedule)
   int* expert_count;
   int* expert_offset;
   int* part_count;
@@ -97,32 +116,24 @@ __device__ __forceinline__ Tile tile_of(const LayoutArgs& a, int b) {
 // shared-memory plan (ints, every array 16-byte aligned)
 // ---------------------------------------------------------------------------
 struct LayoutSmem {
-  int part_s, tot, pre, eoff, pos, scanbuf, cta_hist, red, whist, ewhist, keycnt, keystart, pc,
-      poff, ptot, ppre, pbase, cta_phist, wp, warp_tot, misc, keys, total;
-  __host__ __device__ static int up4(int x) { return (x + 3) & ~3; }
-  __host__ __device__ LayoutSmem(int G, int E, int key_cap) {
-    const int RW = kRedW;
+  int part_s, eoff, pos, scanbuf, row, ctot, cpre, red, whist, kcnt, pc, poff, pbase, wp, misc,
+      keys, total;
+  __host__ __device__ LayoutSmem(int G, int E, int W, int key_cap) {
     int o = 0;
     part_s = o; o += up4(G);
-    tot = o; o += up4(G);
-    pre = o; o += up4(G);
     eoff = o; o += up4(G);
     pos = o; o += up4(G);
     scanbuf = o; o += up4(G);
-    cta_hist = o; o += up4(G);
-    red = o; o += up4(2 * RW);
+    row = o; o += up4(W);
+    ctot = o; o += up4(W);
+    cpre = o; o += up4(W);
+    red = o; o += 2 * kRedW;
     whist = o; o += up4(kLWarps * G);
-    ewhist = o; o += up4(kLWarps * (E + 1));
-    keycnt = o; o += up4(E + 1);
-    keystart = o; o += up4(E + 1);
+    kcnt = o; o += up4(E + 1);
     pc = o; o += up4(E);
     poff = o; o += up4(E + 1);
-    ptot = o; o += up4(E);
-    ppre = o; o += up4(E);
     pbase = o; o += up4(E);
-    cta_phist = o; o += up4(E);
     wp = o; o += up4(kLWarps * E);
-    warp_tot = o; o += up4(kLWarps);
     misc = o; o += 4;
     keys = o; o += up4(key_cap);
     total = o;
@@ -130,15 +141,20 @@ struct LayoutSmem {
 };
 
 struct Smem {
-  int *part_s, *tot, *pre, *eoff, *pos, *scanbuf, *cta_hist, *red, *whist, *ewhist, *keycnt,
-      *keystart, *pc, *poff, *ptot, *ppre, *pbase, *cta_phist, *wp, *warp_tot, *misc, *keys;
-  __device__ Smem(int* sm, const LayoutSmem& P)
-      : part_s(sm + P.part_s), tot(sm + P.tot), pre(sm + P.pre), eoff(sm + P.eoff),
-        pos(sm + P.pos), scanbuf(sm + P.scanbuf), cta_hist(sm + P.cta_hist), red(sm + P.red),
-        whist(sm + P.whist), ewhist(sm + P.ewhist), keycnt(sm + P.keycnt),
-        keystart(sm + P.keystart), pc(sm + P.pc), poff(sm + P.poff), ptot(sm + P.ptot),
-        ppre(sm + P.ppre), pbase(sm + P.pbase), cta_phist(sm + P.cta_phist), wp(sm + P.wp),
-        warp_tot(sm + P.warp_tot), misc(sm + P.misc), keys(sm + P.keys) {}
+  int *part_s, *eoff, *pos, *scanbuf, *row, *ctot, *cpre, *red, *whist, *kcnt, *pc, *poff, *pbase,
+      *wp, *misc, *keys;
+  // views: totals / tile prefixes per expert and per partition
+  int *tot, *pre, *ptot, *ppre;
+  __device__ Smem(int* sm, const LayoutSmem& P, int G)
+      : part_s(sm + P.part_s), eoff(sm + P.eoff), pos(sm + P.pos), scanbuf(sm + P.scanbuf),
+        row(sm + P.row), ctot(sm + P.ctot), cpre(sm + P.cpre), red(sm + P.red),
+        whist(sm + P.whist), kcnt(sm + P.kcnt), pc(sm + P.pc), poff(sm + P.poff),
+        pbase(sm + P.pbase), wp(sm + P.wp), misc(sm + P.misc), keys(sm + P.keys) {
+    tot = ctot;
+    pre = cpre;
+    ptot = ctot + G;
+    ppre = cpre + G;
+  }
 };
 
 // ---------------------------------------------------------------------------
@@ -153,7 +169,8 @@ struct RawIds {
 };
 
 // Fill the shared-memory cache of the tile's ids (16-byte loads when aligned),
-// zero the block's scratch and load the placement map.  Ends with a barrier.
+// zero the block's scratch and load the placement map.  Reads only the
+// caller's inputs.  Ends with a barrier.
 __device__ void stage_tile(const LayoutArgs& a, const Tile& tl, const Smem& S, RawIds& ids) {
   const int tid = threadIdx.x;
   const int* src = a.idx + (size_t)tl.t0 * a.topk;
@@ -176,28 +193,19 @@ __device__ void stage_tile(const LayoutArgs& a, const Tile& tl, const Smem& S, R
   }
   for (int e = tid; e < a.G; e += kLThreads) S.part_s[e] = __ldg(a.part_of + e);
   for (int i = tid; i < kLWarps * a.G; i += kLThreads) S.whist[i] = 0;
-  for (int i = tid; i < kLWarps * (a.E + 1); i += kLThreads) S.ewhist[i] = 0;
+  for (int i = tid; i < a.W; i += kLThreads) S.row[i] = 0;
   for (int p = tid; p < a.E; p += kLThreads) {
     S.pc[p] = 0;
     S.pbase[p] = 0;
-    S.cta_phist[p] = 0;
   }
   if (tid < 4) S.misc[tid] = 0;
   __syncthreads();
 }
 
-// Status bits of the tile (bad expert ids; block `first` also checks the map).
-__device__ int scan_flags(const LayoutArgs& a, const Tile& tl, const Smem& S, const RawIds& ids,
-                          bool first) {
-  int f = 0;
-  for (int i = threadIdx.x; i < tl.n_items; i += kLThreads) {
-    const int e = ids(i);
-    if (e < 0 || e >= a.G) f |= MOE_STATUS_BAD_EXPERT;
-  }
-  if (first)
-    for (int e = threadIdx.x; e < a.G; e += kLThreads)
-      if (!valid_part(S.part_s[e], a.E)) f |= MOE_STATUS_BAD_PART;
-  return f;
+__device__ __forceinline__ int item_key(const LayoutArgs& a, const Smem& S, const RawIds& ids,
+                                        int i) {
+  const int e = ids(i);
+  return (e >= 0 && e < a.G && valid_part(S.part_s[e], a.E)) ? e : -1;
 }
 
 // Per-warp counts of the keys of [0, n) (warp w owns the w-th contiguous
@@ -262,11 +270,11 @@ __device__ void rank_assign(int n, int K, int* whist, KeyOf key_of, OnRank on_ra
   __syncthreads();
 }
 
-// In-place exclusive scan of data[0..n) in shared memory; returns the total.
-__device__ int block_exclusive_scan(int* data, int n, int* warp_tot) {
-  const int tid = threadIdx.x, lane = lane_id(), warp = warp_id();
-  const int ipt = (n + kLThreads - 1) / kLThreads;
-  const int beg = min(n, tid * ipt), end = min(n, beg + ipt);
+// One warp: in-place exclusive scan of data[0..n); returns the total.
+__device__ int warp_exclusive_scan(int* data, int n) {
+  const int lane = lane_id();
+  const int per = (n + kWarp - 1) / kWarp;
+  const int beg = min(n, lane * per), end = min(n, beg + per);
   int s = 0;
   for (int i = beg; i < end; ++i) s += data[i];
   int x = s;
@@ -275,27 +283,43 @@ __device__ int block_exclusive_scan(int* data, int n, int* warp_tot) {
     const int y = __shfl_up_sync(kFull, x, o);
     if (lane >= o) x += y;
   }
-  if (lane == kWarp - 1) warp_tot[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    int v = lane < kLWarps ? warp_tot[lane] : 0;
-#pragma unroll
-    for (int o = 1; o < kWarp; o <<= 1) {
-      const int y = __shfl_up_sync(kFull, v, o);
-      if (lane >= o) v += y;
-    }
-    if (lane < kLWarps) warp_tot[lane] = v;
-  }
-  __syncthreads();
-  int run = x - s + (warp > 0 ? warp_tot[warp - 1] : 0);
+  int run = x - s;
   for (int i = beg; i < end; ++i) {
     const int v = data[i];
     data[i] = run;
     run += v;
   }
-  const int total = warp_tot[kLWarps - 1];
-  __syncthreads();
-  return total;
+  return __shfl_sync(kFull, x, kWarp - 1);
+}
+
+// One warp: position of every expert in (partition, id) order, experts with
+// an invalid placement last.  Reads only the placement map.
+__device__ void expert_order(const LayoutArgs& a, const Smem& S) {
+  const int lane = lane_id(), G = a.G, E = a.E;
+  for (int k = lane; k <= E; k += kWarp) S.kcnt[k] = 0;
+  __syncwarp();
+  const int nbits = key_bits(E + 1);
+  const unsigned lt = lanemask_lt();
+  for (int c = 0; c < G; c += kWarp) {
+    const int e = c + lane;
+    int key = -1;
+    if (e < G) key = valid_part(S.part_s[e], E) ? S.part_s[e] : E;
+    const unsigned peers = match_peers(key, nbits);
+    const int base = key >= 0 ? S.kcnt[key] : 0;
+    __syncwarp();
+    if (key >= 0) {
+      S.pos[e] = base + __popc(peers & lt);  // rank among the experts of its key
+      if (lane == __ffs(peers) - 1) S.kcnt[key] = base + __popc(peers);
+    }
+    __syncwarp();
+  }
+  (void)warp_exclusive_scan(S.kcnt, E + 1);  // start of each key
+  __syncwarp();
+  for (int e = lane; e < G; e += kWarp) {
+    const int key = valid_part(S.part_s[e], E) ? S.part_s[e] : E;
+    S.pos[e] += S.kcnt[key];
+  }
+  __syncwarp();
 }
 
 // Partition bit mask of token tl of the tile (valid pairs only).
@@ -312,63 +336,67 @@ __device__ __forceinline__ unsigned long long token_mask(const LayoutArgs& a, co
   return mask;
 }
 
-// dedup: tokens of the tile holding partition p, into cta_phist[p]
-__device__ void count_tile_parts(const LayoutArgs& a, const Tile& tl, const Smem& S,
-                                 const RawIds& ids) {
-  const int lane = lane_id();
-  for (int r0 = 0; r0 < tl.ntok; r0 += kLThreads) {
-    const int t = r0 + threadIdx.x;
-    const unsigned long long mask = t < tl.ntok ? token_mask(a, ids, S.part_s, t) : 0ull;
-    for (int p = 0; p < a.E; ++p) {
-      const unsigned bal = __ballot_sync(kFull, (mask >> p) & 1ull);
-      if (lane == 0 && bal) atomicAdd(&S.cta_phist[p], __popc(bal));
+// The tile's own row: expert counts (and per-warp bases in whist), with
+// dedup its distinct (token, partition) counts, and the invalid-input
+// counters.  Ends with a barrier.
+__device__ void count_tile(const LayoutArgs& a, const Tile& tl, const Smem& S, const RawIds& ids,
+                           bool first) {
+  const int G = a.G, E = a.E, lane = lane_id();
+  const int fcol = G + (a.dedup ? E : 0);
+  int bad = 0;
+  rank_count(tl.n_items, G, S.whist, S.row, [&](int i) {
+    const int e = ids(i);
+    bad += (e < 0 || e >= G);
+    return (e >= 0 && e < G && valid_part(S.part_s[e], E)) ? e : -1;
+  });
+  int badp = 0;
+  if (first)
+    for (int e = threadIdx.x; e < G; e += kLThreads) badp += !valid_part(S.part_s[e], E);
+  if (bad) atomicAdd(&S.row[fcol], bad);
+  if (badp) atomicAdd(&S.row[fcol + 1], badp);
+  if (a.dedup) {
+    for (int r0 = 0; r0 < tl.ntok; r0 += kLThreads) {
+      const int t = r0 + threadIdx.x;
+      const unsigned long long mask = t < tl.ntok ? token_mask(a, ids, S.part_s, t) : 0ull;
+      for (int p = 0; p < E; ++p) {
+        const unsigned bal = __ballot_sync(kFull, (mask >> p) & 1ull);
+        if (lane == 0 && bal) atomicAdd(&S.row[G + p], __popc(bal));
+      }
     }
   }
   __syncthreads();
 }
 
-// expert order (partition, id) -> pos[e]; offsets eoff[e], partition counts
-// and offsets.  Needs tot[] (and ptot[] with dedup).  Returns R_exp.
+// expert offsets (needs pos[], tot[]), partition counts and offsets (needs
+// ptot[] with dedup).  Returns R_exp.  Ends with a barrier.
 __device__ int finish_offsets(const LayoutArgs& a, const Smem& S) {
   const int G = a.G, E = a.E, tid = threadIdx.x;
-  auto ekey = [&](int e) {
-    const int p = S.part_s[e];
-    return valid_part(p, E) ? p : E;
-  };
-  rank_count(G, E + 1, S.ewhist, S.keycnt, ekey);
-  if (tid == 0) {
-    int run = 0;
-    for (int k = 0; k <= E; ++k) {
-      S.keystart[k] = run;
-      run += S.keycnt[k];
-    }
-  }
-  __syncthreads();
-  rank_assign(
-      G, E + 1, S.ewhist, ekey, [&](int e, int k, int r) { S.pos[e] = S.keystart[k] + r; },
-      [](int) {});
-  for (int e = tid; e < G; e += kLThreads) S.scanbuf[S.pos[e]] = S.tot[e];
-  __syncthreads();
-  const int R_exp = block_exclusive_scan(S.scanbuf, G, S.warp_tot);
   for (int e = tid; e < G; e += kLThreads) {
-    S.eoff[e] = S.scanbuf[S.pos[e]];
+    S.scanbuf[S.pos[e]] = S.tot[e];
     if (!a.dedup && valid_part(S.part_s[e], E) && S.tot[e]) atomicAdd(&S.pc[S.part_s[e]], S.tot[e]);
   }
   __syncthreads();
-  if (tid == 0) {
-    int run = 0;
-    for (int p = 0; p < E; ++p) {
-      if (a.dedup) S.pc[p] = S.ptot[p];
-      S.poff[p] = run;
-      run += S.pc[p];
+  if (warp_id() == 0) {
+    const int R_exp = warp_exclusive_scan(S.scanbuf, G);
+    if (a.dedup)
+      for (int p = lane_id(); p < E; p += kWarp) S.pc[p] = S.ptot[p];
+    __syncwarp();
+    for (int p = lane_id(); p < E; p += kWarp) S.poff[p] = S.pc[p];
+    __syncwarp();
+    const int R_disp = warp_exclusive_scan(S.poff, E);
+    if (lane_id() == 0) {
+      S.poff[E] = R_disp;
+      S.misc[2] = R_exp;
     }
-    S.poff[E] = run;
   }
   __syncthreads();
-  return R_exp;
+  for (int e = tid; e < G; e += kLThreads) S.eoff[e] = S.scanbuf[S.pos[e]];
+  __syncthreads();
+  return S.misc[2];
 }
 
-__device__ void write_globals(const LayoutArgs& a, const Smem& S, int R_exp, int flags) {
+__device__ void write_globals(const LayoutArgs& a, const Smem& S, int R_exp) {
+  const int fcol = a.G + (a.dedup ? a.E : 0);
   for (int e = threadIdx.x; e < a.G; e += kLThreads) {
     a.expert_count[e] = S.tot[e];
     a.expert_offset[e] = S.eoff[e];
@@ -380,7 +408,8 @@ __device__ void write_globals(const LayoutArgs& a, const Smem& S, int R_exp, int
   if (threadIdx.x == 0) {
     a.expert_offset[a.G] = R_exp;
     a.part_offset[a.E] = S.poff[a.E];
-    *a.status = flags;
+    *a.status = (S.ctot[fcol] > 0 ? MOE_STATUS_BAD_EXPERT : 0) |
+                (S.ctot[fcol + 1] > 0 ? MOE_STATUS_BAD_PART : 0);
   }
 }
 
@@ -429,12 +458,8 @@ __device__ void rank_tile_items(const LayoutArgs& a, const Tile& tl, const Smem&
                                 const RawIds& ids) {
   const int G = a.G, E = a.E;
   int* exp_row = a.exp_row + (size_t)tl.t0 * a.topk;
-  auto ikey = [&](int i) {
-    const int e = ids(i);
-    return (e >= 0 && e < G && valid_part(S.part_s[e], E)) ? e : -1;
-  };
   rank_assign(
-      tl.n_items, G, S.whist, ikey,
+      tl.n_items, G, S.whist, [&](int i) { return item_key(a, S, ids, i); },
       [&](int i, int e, int r) {
         const int row = S.eoff[e] + S.pre[e] + r;
         exp_row[i] = row;
@@ -448,20 +473,15 @@ __device__ void rank_tile_items(const LayoutArgs& a, const Tile& tl, const Smem&
       [&](int i) { exp_row[i] = -1; });
 }
 
-__device__ __forceinline__ int item_key(const LayoutArgs& a, const Smem& S, const RawIds& ids,
-                                        int i) {
-  const int e = ids(i);
-  return (e >= 0 && e < a.G && valid_part(S.part_s[e], a.E)) ? e : -1;
-}
-
 // ---------------------------------------------------------------------------
-// schedule 1: one cluster
+// schedule 1: one cluster of gridDim.x blocks
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kLThreads) layout_cluster_kernel(LayoutArgs a) {
   extern __shared__ __align__(16) int sm[];
   cg::cluster_group cluster = cg::this_cluster();
-  const LayoutSmem P(a.G, a.E, a.key_cap);
-  const Smem S(sm, P);
+  const LayoutSmem P(a.G, a.E, a.W, a.key_cap);
+  const Smem S(sm, P, a.G);
+  const int C = (int)cluster.num_blocks();
   const int r = (int)cluster.block_rank();
   const int tid = threadIdx.x;
   const Tile tl = tile_of(a, r);
@@ -469,50 +489,31 @@ __global__ void __launch_bounds__(kLThreads) layout_cluster_kernel(LayoutArgs a)
   pdl_trigger();
   RawIds ids;
   stage_tile(a, tl, S, ids);
-
-  // count the tile; the per-warp bases stay in whist for the ranks below
-  const int f = scan_flags(a, tl, S, ids, r == 0);
-  if (f) atomicOr(&S.misc[0], f);
-  rank_count(tl.n_items, a.G, S.whist, S.cta_hist, [&](int i) { return item_key(a, S, ids, i); });
-  if (a.dedup) count_tile_parts(a, tl, S, ids);
+  count_tile(a, tl, S, ids, r == 0);
+  if (warp_id() == 0) expert_order(a, S);
   cluster.sync();
 
   // exchange: totals over the cluster and the prefix of the tiles before r
-  for (int e = tid; e < a.G; e += kLThreads) {
-    int v[kClusterCTAs];
+  for (int c = tid; c < a.W; c += kLThreads) {
+    int v[kMaxCluster];
 #pragma unroll
-    for (int q = 0; q < kClusterCTAs; ++q) v[q] = cluster.map_shared_rank(S.cta_hist, q)[e];
+    for (int q = 0; q < kMaxCluster; ++q) v[q] = q < C ? cluster.map_shared_rank(S.row, q)[c] : 0;
     int all = 0, bef = 0;
 #pragma unroll
-    for (int q = 0; q < kClusterCTAs; ++q) {
+    for (int q = 0; q < kMaxCluster; ++q) {
       all += v[q];
       bef += q < r ? v[q] : 0;
     }
-    S.tot[e] = all;
-    S.pre[e] = bef;
+    S.ctot[c] = all;
+    S.cpre[c] = bef;
   }
-  if (a.dedup) {
-    for (int p = tid; p < a.E; p += kLThreads) {
-      int all = 0, bef = 0;
-      for (int q = 0; q < kClusterCTAs; ++q) {
-        const int v = cluster.map_shared_rank(S.cta_phist, q)[p];
-        all += v;
-        bef += q < r ? v : 0;
-      }
-      S.ptot[p] = all;
-      S.ppre[p] = bef;
-    }
-  }
-  int flags = 0;
-  if (r == 0 && tid < kClusterCTAs) flags = cluster.map_shared_rank(S.misc, tid)[0];
   __syncthreads();
-  if (r == 0 && flags) atomicOr(&S.misc[1], flags);
 
   const int R_exp = finish_offsets(a, S);
-  if (r == 0) write_globals(a, S, R_exp, S.misc[1]);
+  if (r == 0) write_globals(a, S, R_exp);
   if (a.dedup) rank_tile_parts(a, tl, S, ids);
   rank_tile_items(a, tl, S, ids);
-  cluster.sync();  // no block leaves while another may still read its histograms
+  cluster.sync();  // no block leaves while another may still read its row
 }
 
 // ---------------------------------------------------------------------------
@@ -520,116 +521,76 @@ __global__ void __launch_bounds__(kLThreads) layout_cluster_kernel(LayoutArgs a)
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kLThreads) layout_count_kernel(LayoutArgs a) {
   extern __shared__ __align__(16) int sm[];
-  const LayoutSmem P(a.G, a.E, a.key_cap);
-  const Smem S(sm, P);
+  const LayoutSmem P(a.G, a.E, a.W, a.key_cap);
+  const Smem S(sm, P, a.G);
   const int b = blockIdx.x;
   const Tile tl = tile_of(a, b);
   pdl_wait();
   pdl_trigger();
   RawIds ids;
   stage_tile(a, tl, S, ids);
-  const int f = scan_flags(a, tl, S, ids, b == 0);
-  if (f) atomicOr(&S.misc[0], f);
-  rank_count(tl.n_items, a.G, S.whist, S.cta_hist, [&](int i) { return item_key(a, S, ids, i); });
-  if (a.dedup) count_tile_parts(a, tl, S, ids);
-  int* th = a.tile_hist + (size_t)b * a.G;
-  for (int i = threadIdx.x; i < a.G; i += kLThreads) th[i] = S.cta_hist[i];
-  if (a.dedup)
-    for (int i = threadIdx.x; i < a.E; i += kLThreads)
-      a.tile_phist[(size_t)b * a.E + i] = S.cta_phist[i];
-  if (threadIdx.x == 0) a.tile_flags[b] = S.misc[0];
+  count_tile(a, tl, S, ids, b == 0);
+  int4* dst = reinterpret_cast<int4*>(a.tile_rows + (size_t)b * a.W);
+  const int4* src = reinterpret_cast<const int4*>(S.row);
+  for (int i = threadIdx.x; i < (a.W >> 2); i += kLThreads) dst[i] = src[i];
 }
 
-// Column sums of a [rows][cols] int matrix in global memory (L2): total over
-// all rows and over rows < b.  Each thread keeps up to 8 16-byte loads in
-// flight.  `red` holds 2 * kRedW ints (cols <= MOE_MAX_G <= kRedW).
-__device__ void column_sums(const int* src, int rows, int cols, int b, int* red, int* total,
+// Column sums of the [rows][W] tile rows in global memory (L2): total over
+// all rows and over rows < b, with up to 8 16-byte loads in flight per
+// thread.  W is a multiple of 4 and at most kRedW.
+__device__ void column_sums(const int* src, int rows, int W, int b, int* red, int* total,
                             int* before) {
   const int tid = threadIdx.x;
-  const int RW = kRedW;
-  const bool vec = (cols & 3) == 0 && (reinterpret_cast<uintptr_t>(src) & 15) == 0;
-  if (vec) {
-    const int C4 = cols >> 2;
-    const int S = C4 <= kLThreads ? kLThreads / C4 : 1;
-    for (int slot = tid; slot < C4 * S; slot += kLThreads) {
-      const int c4 = slot % C4, s = slot / C4;
-      int4 all = make_int4(0, 0, 0, 0), bef = all;
+  const int C4 = W >> 2;
+  const int S = C4 <= kLThreads ? kLThreads / C4 : 1;
+  for (int slot = tid; slot < C4 * S; slot += kLThreads) {
+    const int c4 = slot % C4, s = slot / C4;
+    int4 all = make_int4(0, 0, 0, 0), bef = all;
 #pragma unroll 8
-      for (int r = s; r < rows; r += S) {
-        const int4 v = __ldcg(reinterpret_cast<const int4*>(src + (size_t)r * cols) + c4);
-        all.x += v.x; all.y += v.y; all.z += v.z; all.w += v.w;
-        if (r < b) {
-          bef.x += v.x; bef.y += v.y; bef.z += v.z; bef.w += v.w;
-        }
+    for (int r = s; r < rows; r += S) {
+      const int4 v = __ldcg(reinterpret_cast<const int4*>(src + (size_t)r * W) + c4);
+      all.x += v.x; all.y += v.y; all.z += v.z; all.w += v.w;
+      if (r < b) {
+        bef.x += v.x; bef.y += v.y; bef.z += v.z; bef.w += v.w;
       }
-      const int base = s * cols + 4 * c4;
-      red[base] = all.x; red[base + 1] = all.y; red[base + 2] = all.z; red[base + 3] = all.w;
-      red[RW + base] = bef.x; red[RW + base + 1] = bef.y;
-      red[RW + base + 2] = bef.z; red[RW + base + 3] = bef.w;
     }
-    __syncthreads();
-    for (int c = tid; c < cols; c += kLThreads) {
-      int all = 0, bef = 0;
-      for (int s = 0; s < S; ++s) {
-        all += red[s * cols + c];
-        bef += red[RW + s * cols + c];
-      }
-      total[c] = all;
-      before[c] = bef;
+    const int base = s * W + 4 * c4;
+    red[base] = all.x; red[base + 1] = all.y; red[base + 2] = all.z; red[base + 3] = all.w;
+    red[kRedW + base] = bef.x; red[kRedW + base + 1] = bef.y;
+    red[kRedW + base + 2] = bef.z; red[kRedW + base + 3] = bef.w;
+  }
+  __syncthreads();
+  for (int c = tid; c < W; c += kLThreads) {
+    int all = 0, bef = 0;
+    for (int s = 0; s < S; ++s) {
+      all += red[s * W + c];
+      bef += red[kRedW + s * W + c];
     }
-  } else {
-    const int S = cols <= kLThreads ? kLThreads / cols : 1;
-    for (int slot = tid; slot < cols * S; slot += kLThreads) {
-      const int c = slot % cols, s = slot / cols;
-      int all = 0, bef = 0;
-#pragma unroll 8
-      for (int r = s; r < rows; r += S) {
-        const int v = __ldcg(src + (size_t)r * cols + c);
-        all += v;
-        bef += (r < b) ? v : 0;
-      }
-      red[slot] = all;
-      red[RW + slot] = bef;
-    }
-    __syncthreads();
-    for (int c = tid; c < cols; c += kLThreads) {
-      int all = 0, bef = 0;
-      for (int s = 0; s < S; ++s) {
-        all += red[s * cols + c];
-        bef += red[RW + s * cols + c];
-      }
-      total[c] = all;
-      before[c] = bef;
-    }
+    total[c] = all;
+    before[c] = bef;
   }
   __syncthreads();
 }
 
 __global__ void __launch_bounds__(kLThreads) layout_rank_kernel(LayoutArgs a) {
   extern __shared__ __align__(16) int sm[];
-  const LayoutSmem P(a.G, a.E, a.key_cap);
-  const Smem S(sm, P);
+  const LayoutSmem P(a.G, a.E, a.W, a.key_cap);
+  const Smem S(sm, P, a.G);
   const int b = blockIdx.x;
   const Tile tl = tile_of(a, b);
-  // the caller's inputs were complete before layout_count_kernel started,
-  // so they are staged before waiting for its histograms
+  // Everything that depends only on the caller's inputs -- which were
+  // complete before layout_count_kernel started -- runs before the wait:
+  // the tile's ids, its per-warp counts and the expert order.
   RawIds ids;
   stage_tile(a, tl, S, ids);
+  rank_count(tl.n_items, a.G, S.whist, nullptr, [&](int i) { return item_key(a, S, ids, i); });
+  if (warp_id() == 0) expert_order(a, S);
   pdl_wait();
   pdl_trigger();
 
-  column_sums(a.tile_hist, a.n_tiles, a.G, b, S.red, S.tot, S.pre);
-  if (a.dedup) column_sums(a.tile_phist, a.n_tiles, a.E, b, S.red, S.ptot, S.ppre);
-  rank_count(tl.n_items, a.G, S.whist, nullptr, [&](int i) { return item_key(a, S, ids, i); });
-
+  column_sums(a.tile_rows, a.n_tiles, a.W, b, S.red, S.ctot, S.cpre);
   const int R_exp = finish_offsets(a, S);
-  if (b == 0) {
-    int f = 0;
-    for (int q = threadIdx.x; q < a.n_tiles; q += kLThreads) f |= __ldcg(a.tile_flags + q);
-    if (f) atomicOr(&S.misc[1], f);
-    __syncthreads();
-    write_globals(a, S, R_exp, S.misc[1]);
-  }
+  if (b == 0) write_globals(a, S, R_exp);
   if (a.dedup) rank_tile_parts(a, tl, S, ids);
   rank_tile_items(a, tl, S, ids);
 }
@@ -637,7 +598,8 @@ __global__ void __launch_bounds__(kLThreads) layout_rank_kernel(LayoutArgs a) {
 bool use_cluster(const moe_problem_t& p) { return (int64_t)p.M * p.topk <= kClusterItems; }
 
 size_t smem_bytes(const moe_problem_t& p, int key_cap) {
-  return sizeof(int) * (size_t)LayoutSmem(p.G, p.E_part, key_cap).total;
+  const int W = row_width(p.G, p.E_part, p.dedup);
+  return sizeof(int) * (size_t)LayoutSmem(p.G, p.E_part, W, key_cap).total;
 }
 
 }  // namespace
@@ -654,8 +616,7 @@ int layout_num_tiles(int M) {
 }
 
 size_t layout_workspace_bytes(const moe_problem_t& p) {
-  const size_t nt = (size_t)layout_num_tiles(p.M);
-  const size_t ints = nt * ((size_t)p.G + (p.dedup ? (size_t)p.E_part : 0) + 1);
+  const size_t ints = (size_t)layout_num_tiles(p.M) * row_width(p.G, p.E_part, p.dedup);
   return (ints * sizeof(int) + 255) / 256 * 256;
 }
 
@@ -668,6 +629,7 @@ cudaError_t launch_layout(const moe_problem_t& p, const int32_t* topk_idx,
   a.topk = p.topk;
   a.E = p.E_part;
   a.dedup = p.dedup;
+  a.W = row_width(p.G, p.E_part, p.dedup);
   a.idx = topk_idx;
   a.part_of = part_of;
   a.expert_count = lay.expert_count;
@@ -681,22 +643,25 @@ cudaError_t launch_layout(const moe_problem_t& p, const int32_t* topk_idx,
   a.status = lay.status;
 
   if (use_cluster(p)) {
+    const int items = p.M * p.topk;
+    const int C = std::min(kMaxCluster, std::max(1, (items + MOE_CLUSTER_BLOCK_ITEMS - 1) /
+                                                        MOE_CLUSTER_BLOCK_ITEMS));
     // tiles of a multiple of 4 tokens keep every tile's ids 16-byte aligned
-    a.T = std::max(4, ((p.M + kClusterCTAs - 1) / kClusterCTAs + 3) / 4 * 4);
-    a.n_tiles = kClusterCTAs;
+    a.T = std::max(4, ((p.M + C - 1) / C + 3) / 4 * 4);
+    a.n_tiles = C;
     a.key_cap = a.T * p.topk;
-    a.tile_hist = a.tile_phist = a.tile_flags = nullptr;
+    a.tile_rows = nullptr;
     const size_t smem = smem_bytes(p, a.key_cap);
     cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void*>(layout_cluster_kernel), smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(kClusterCTAs);
+    cfg.gridDim = dim3(C);
     cfg.blockDim = dim3(kLThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = kClusterCTAs;
+    attr[0].val.clusterDim.x = C;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -711,10 +676,7 @@ cudaError_t launch_layout(const moe_problem_t& p, const int32_t* topk_idx,
   a.T = layout_tile_tokens(p.M);
   a.n_tiles = layout_num_tiles(p.M);
   a.key_cap = a.T * p.topk <= kMaxTileItems ? a.T * p.topk : 0;
-  int* ws = static_cast<int*>(workspace);
-  a.tile_hist = ws;
-  a.tile_phist = ws + (size_t)a.n_tiles * p.G;
-  a.tile_flags = a.tile_phist + (p.dedup ? (size_t)a.n_tiles * p.E_part : 0);
+  a.tile_rows = static_cast<int*>(workspace);
   const size_t smem = smem_bytes(p, a.key_cap);
   cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void*>(layout_count_kernel), smem);
   if (e != cudaSuccess) return e;

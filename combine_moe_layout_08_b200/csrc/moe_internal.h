@@ -45,8 +45,8 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // least `bytes` (once per device and kernel; no-op up to 48 KB).
 cudaError_t allow_dynamic_smem(const void* kernel, size_t bytes);
 
-// Tokens per layout tile: about one tile per SM, at least 64 tokens, a
-// multiple of 32.
+// Tokens per layout tile: about one tile per SM, at least
+// MOE_TILE_MIN_TOKENS, a multiple of 32 (so at most 148 tiles).
 int layout_tile_tokens(int M);
 int layout_num_tiles(int M);
 size_t layout_workspace_bytes(const moe_problem_t& p);

@@ -161,9 +161,9 @@ int moe_layout(const moe_problem_t *prob, const int32_t *topk_idx,
  *   library, held by every GPU that loads it until the process exits.
  *   Limit: a problem whose moe_layout_workspace_size() exceeds
  *   MOE_STATIC_SCRATCH_BYTES is rejected with MOE_ERR_WORKSPACE before any
- *   launch.  The layout uses at most 148 tiles, so every M fits when
- *   G + E_part <= 441 (G = 256, E_part = 8 always fits); larger G fit only
- *   for small M.
+ *   launch.  The layout uses at most 148 tiles of G + E_part + 2 ints each
+ *   (padded to 4), so every M fits when G + E_part <= 438 (G = 256,
+ *   E_part = 8 always fits); larger G fit only for small M.
  *   The first call on a device looks up the array's device address (one
  *   cudaGetSymbolAddress with that device current); make it before any
  *   stream capture.  Every call shares the array: calls whose execution

@@ -67,10 +67,12 @@ def test_workspace_size(L):
     assert ws > 0 and ws % 256 == 0
     big = L.moe_layout_workspace_size(ctypes.byref(P(M=65536, dedup=1)))
     assert big > ws
-    # per-tile histograms, one tile per SM-sized token slice
-    T = max(64, ((65536 + 147) // 148 + 31) // 32 * 32)
+    # one row per tile (about one tile per SM): G expert counts, E partition
+    # counts (dedup), two invalid-input counters, padded to 4 ints
+    T = max(128, ((65536 + 147) // 148 + 31) // 32 * 32)
     nt = (65536 + T - 1) // T
-    assert big == ((nt * (256 + 8 + 1) * 4 + 255) // 256) * 256
+    W = (256 + 8 + 2 + 3) // 4 * 4
+    assert big == ((nt * W * 4 + 255) // 256) * 256
     for bad in (P(N=7), P(G=0), P(G=1025), P(topk=0), P(topk=33), P(E_part=0), P(E_part=65),
                 P(M=-1), P(fp8=1, N=7176), P(dedup=2), P(M=1 << 28, topk=8)):
         assert L.moe_layout_workspace_size(ctypes.byref(bad)) == 0
