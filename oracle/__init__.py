@@ -14,7 +14,10 @@ Each function follows a passage of the pages:
 * :func:`dispatch` -- issue #117 all_to_all_kernel arguments (row copy with
   optional scales, ``WITH_SCALE``), FP8 e4m3 per 128 columns;
 * :func:`combine` -- Purlin section 3.3, SCORE (exclusive ownership, ordered
-  accumulation).
+  accumulation);
+* :func:`combine_partial` / :func:`combine_reduce` -- the two-level combine
+  of a deduplicated dispatch: per (token, partition) reduce in slot order,
+  then the token's sum over partitions in partition order.
 
 Pins (tests/test_oracle_*.py): pure-Python brute force of the layout
 definition on every tiny input, layout invariants, the e4m3 encoder against a
@@ -60,6 +63,10 @@ def lib():
         L.oracle_combine.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int64,
                                      ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                      ctypes.c_void_p, ctypes.c_void_p]
+        L.oracle_combine_partial.restype = ctypes.c_int
+        L.oracle_combine_partial.argtypes = [ctypes.c_int32] * 4 + [ctypes.c_int64] + [ctypes.c_void_p] * 8
+        L.oracle_combine_reduce.restype = ctypes.c_int
+        L.oracle_combine_reduce.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int64] + [ctypes.c_void_p] * 4
         _lib = L
     return _lib
 
@@ -158,6 +165,49 @@ def combine(y_bits, topk_weights, exp_row, tokens=None):
     return out
 
 
+def combine_partial(y_bits, topk_weights, topk_idx, part_of, lay, tokens=None):
+    """Partition-side reduce of the two-level (dedup) combine: bf16 bits
+    [R_disp, N] in dispatch-row space (rows of tokens not listed stay 0)."""
+    y = _c(y_bits, np.uint16)
+    N = y.shape[1]
+    w = _c(topk_weights, np.float32)
+    idx = _c(topk_idx, np.int32)
+    M, topk = idx.shape
+    po = _c(part_of, np.int32)
+    er = _c(lay["exp_row"], np.int32)
+    dr = _c(lay["disp_row"], np.int32)
+    E = dr.shape[1]
+    z = np.zeros((max(lay["R_disp"], 1), N), np.uint16)
+    if tokens is None:
+        n_tok, tk = M, None
+    else:
+        tk = _c(tokens, np.int64)
+        n_tok = tk.shape[0]
+    rc = lib().oracle_combine_partial(N, topk, E, po.shape[0], n_tok, _p(tk), _p(idx), _p(po),
+                                      _p(y), _p(w), _p(er), _p(dr), _p(z))
+    if rc != 0:
+        raise MemoryError("oracle_combine_partial: host allocation failed")
+    return z[:lay["R_disp"]]
+
+
+def combine_reduce(z_bits, disp_row, tokens=None):
+    """Token-side sum of the two-level combine over partitions (p order)."""
+    z = _c(z_bits, np.uint16)
+    N = z.shape[1]
+    dr = _c(disp_row, np.int32)
+    M, E = dr.shape
+    if tokens is None:
+        n_tok, tk = M, None
+    else:
+        tk = _c(tokens, np.int64)
+        n_tok = tk.shape[0]
+    out = np.zeros((n_tok, N), np.uint16)
+    rc = lib().oracle_combine_reduce(N, E, n_tok, _p(tk), _p(z), _p(dr), _p(out))
+    if rc != 0:
+        raise MemoryError("oracle_combine_reduce: host allocation failed")
+    return out
+
+
 def bf16_round(values) -> np.ndarray:
     """float32 -> bf16 bits (uint16), nearest-even."""
     v = _c(values, np.float32).ravel()
@@ -193,7 +243,8 @@ def bits_to_f32(b) -> np.ndarray:
     return (np.asarray(b, np.uint32) << 16).view(np.float32)
 
 
-__all__ = ["layout", "dispatch", "combine", "bf16_round", "e4m3_encode", "step",
+__all__ = ["layout", "dispatch", "combine", "combine_partial", "combine_reduce",
+           "bf16_round", "e4m3_encode", "step",
            "bf16_bits", "bits_to_f32", "STATUS_BAD_EXPERT", "STATUS_BAD_PART",
            "lib"]
 

@@ -359,3 +359,78 @@ int oracle_combine(int32_t N, int32_t topk, int64_t n_tok,
     free(acc);
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* two-level combine (dedup return path)                                    */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * With per-partition dedup a token was sent once per partition; on the way
+ * back each partition first reduces the outputs of the token's experts it
+ * holds (Zyphra news item: one copy per GPU; Purlin section 3.3, SCORE:
+ * ordered accumulation), then the token's owner sums the partitions.
+ *
+ * Partition side: for every dispatch row r = disp_row[t, p],
+ *   z[r, c] = bf16( fma chain over k = 0..topk-1 with part_of[idx[t,k]] = p
+ *                   of w[t,k] * y[exp_row[t,k], c], from +0 )
+ * Token side:
+ *   out[t, c] = bf16( sum over p = 0..E_part-1 with disp_row[t,p] >= 0 of
+ *                     float(z[disp_row[t,p], c]), fp32 additions from +0 )
+ * Pairs left out by the layout (exp_row = -1) contribute nothing.
+ *
+ * oracle_combine_partial writes z rows (uint16 bf16 bits) in dispatch-row
+ * space for the tokens tokens[0..n_tok) (NULL: all M); z has R rows.
+ * Returns 0, or -1 when a host allocation fails.
+ */
+int oracle_combine_partial(int32_t N, int32_t topk, int32_t E_part, int32_t G,
+                           int64_t n_tok, const int64_t *tokens,
+                           const int32_t *topk_idx, const int32_t *part_of,
+                           const uint16_t *y, const float *w,
+                           const int32_t *exp_row, const int32_t *disp_row,
+                           uint16_t *z)
+{
+    float *acc = (float *)malloc(sizeof(float) * (size_t)(N > 0 ? N : 1));
+    if (!acc) return -1;
+    for (int64_t i = 0; i < n_tok; ++i) {
+        int64_t t = tokens ? tokens[i] : i;
+        for (int32_t p = 0; p < E_part; ++p) {
+            int32_t r = disp_row[t * E_part + p];
+            if (r < 0) continue;
+            for (int32_t c = 0; c < N; ++c) acc[c] = 0.0f;
+            for (int32_t k = 0; k < topk; ++k) {
+                int32_t er = exp_row[t * topk + k];
+                int32_t e = topk_idx[t * topk + k];
+                if (er < 0 || e < 0 || e >= G || part_of[e] != p) continue;
+                float wk = w[t * topk + k];
+                const uint16_t *yr = y + (int64_t)er * N;
+                for (int32_t c = 0; c < N; ++c)
+                    acc[c] = fmaf(wk, orc_bf16_to_f32(yr[c]), acc[c]);
+            }
+            for (int32_t c = 0; c < N; ++c) z[(int64_t)r * N + c] = orc_f32_to_bf16(acc[c]);
+        }
+    }
+    free(acc);
+    return 0;
+}
+
+/* out row i = token tokens[i] (NULL: token i) summed over its partitions */
+int oracle_combine_reduce(int32_t N, int32_t E_part, int64_t n_tok,
+                          const int64_t *tokens, const uint16_t *z,
+                          const int32_t *disp_row, uint16_t *out)
+{
+    float *acc = (float *)malloc(sizeof(float) * (size_t)(N > 0 ? N : 1));
+    if (!acc) return -1;
+    for (int64_t i = 0; i < n_tok; ++i) {
+        int64_t t = tokens ? tokens[i] : i;
+        for (int32_t c = 0; c < N; ++c) acc[c] = 0.0f;
+        for (int32_t p = 0; p < E_part; ++p) {
+            int32_t r = disp_row[t * E_part + p];
+            if (r < 0) continue;
+            const uint16_t *zr = z + (int64_t)r * N;
+            for (int32_t c = 0; c < N; ++c) acc[c] = acc[c] + orc_bf16_to_f32(zr[c]);
+        }
+        for (int32_t c = 0; c < N; ++c) out[i * N + c] = orc_f32_to_bf16(acc[c]);
+    }
+    free(acc);
+    return 0;
+}

@@ -47,6 +47,13 @@ MUTANTS = [
     ("combine gate sign", "int oracle_combine", "acc[c] = fmaf(wk,", "acc[c] = fmaf(-wk,"),
     ("combine token row", "int oracle_combine", "y + (int64_t)r * N", "y + (int64_t)t * N"),
     ("dispatch wrong row", "void oracle_dispatch", "x + (int64_t)disp_token[r] * N", "x + (int64_t)r * N"),
+    ("partial: wrong partition test", "int oracle_combine_partial", "part_of[e] != p", "part_of[e] == p"),
+    ("partial: drops last slot", "int oracle_combine_partial", "for (int32_t k = 0; k < topk; ++k)",
+     "for (int32_t k = 0; k < topk - 1; ++k)"),
+    ("partial: gate sign", "int oracle_combine_partial", "acc[c] = fmaf(wk,", "acc[c] = fmaf(-wk,"),
+    ("reduce: drops first partition", "int oracle_combine_reduce", "for (int32_t p = 0; p < E_part; ++p)",
+     "for (int32_t p = 1; p < E_part; ++p)"),
+    ("reduce: wrong row", "int oracle_combine_reduce", "z + (int64_t)r * N", "z + (int64_t)t * N"),
 ]
 
 
@@ -72,6 +79,9 @@ def _pins():
         lambda: C.test_combine_one_hot_identity(3),
         lambda: C.test_combine_uniform_gates_identity(4),
         lambda: C.test_combine_within_fp64_bound(5),
+        lambda: C.test_two_level_one_hot_identity(4),
+        lambda: C.test_two_level_colocated_uniform_identity(4),
+        lambda: C.test_two_level_within_fp64_bounds(5, 3),
     ]
 
 
