@@ -50,7 +50,7 @@ L2_FLUSH_BYTES = 256 << 20
 # ---------------------------------------------------------------------------
 # algorithmic bytes (HBM traffic the path cannot avoid), per kernel
 # ---------------------------------------------------------------------------
-def algorithmic_bytes(w: W.Workload, R_exp: int, R_disp: int) -> dict:
+def algorithmic_bytes(w: W.Workload, R_exp: int, R_disp: int, two_level: bool = False) -> dict:
     M, N, G, k, E = w.M, w.N, w.G, w.topk, w.E_part
     layout = 4 * M * k + 4 * G + 4 * M * k + 4 * R_disp + 4 * (2 * G + 2 * E + 2)
     if w.dedup:
@@ -58,6 +58,13 @@ def algorithmic_bytes(w: W.Workload, R_exp: int, R_disp: int) -> dict:
     s = 1 if w.fp8 else 2
     dispatch = 2 * M * N + R_disp * N * s + (4 * R_disp * (N // 128) if w.fp8 else 0)
     dispatch += 4 * M * (E if w.dedup else k)
+    if two_level:
+        # partition side: gather the expert rows, write one row per (token, partition);
+        # token side: read those rows back, write the token rows
+        partial = 2 * R_exp * N + 2 * R_disp * N + 8 * M * k + 4 * R_exp
+        reduce = 2 * R_disp * N + 2 * M * N + 4 * M * E
+        return {"layout": layout, "dispatch": dispatch, "combine_partial": partial,
+                "combine_reduce": reduce}
     combine = 2 * R_exp * N + 2 * M * N + 8 * M * k
     return {"layout": layout, "dispatch": dispatch, "combine": combine}
 
@@ -279,11 +286,15 @@ def run_ours(args, w):
     # external events between the kernels
     with torch.cuda.stream(stream):
         for _ in range(3):
-            buf.step(idx, po, x, y, gates)
+            buf.step(idx, po, x, y, gates, two_level=args.combine == "two-level")
     stream.synchronize()
+    two_level = args.combine == "two-level"
+    if two_level and not w.dedup:
+        raise SystemExit("--combine two-level needs a dedup workload")
     # events inside the graph bracket the step's kernels on the device (the
     # graph's own launch latency, which back-to-back steps hide, stays out)
-    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+    names = ["layout", "dispatch"] + (["combine_partial", "combine_reduce"] if two_level else ["combine"])
+    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(names) + 1)]
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
         ev[0].record()
@@ -291,14 +302,20 @@ def run_ours(args, w):
         ev[1].record()
         buf.dispatch_(x)
         ev[2].record()
-        buf.combine_(y, gates)
+        if two_level:
+            buf.combine_two_level_(y, gates)  # two kernels: events only around the pair
+        else:
+            buf.combine_(y, gates)
         ev[3].record()
     R_exp = int(buf.layout.expert_offset[w.G].item())
     R_disp = int(buf.layout.part_offset[w.E_part].item())
     status = int(buf.layout.status.item())
     if status:
         raise SystemExit(f"layout status {status}")
-    abytes = algorithmic_bytes(wr, R_exp, R_disp)
+    abytes = algorithmic_bytes(wr, R_exp, R_disp, two_level)
+    if two_level:  # one timed interval covers both combine kernels
+        abytes = {"layout": abytes["layout"], "dispatch": abytes["dispatch"],
+                  "combine": abytes["combine_partial"] + abytes["combine_reduce"]}
     step_bytes = sum(abytes.values())
 
     def timed_step():
@@ -327,7 +344,8 @@ def run_ours(args, w):
                "combine": float(per[:, 3].mean())}
 
     # end to end through the public API with host buffers
-    e2e = run_e2e(args, wr, buf, idx_h, po_h, g_h, x, y, stream, dev, flush, step_bytes)
+    e2e = run_e2e(args, wr, buf, idx_h, po_h, g_h, x, y, stream, dev, flush, step_bytes,
+                  two_level)
 
     # aggregate over ranks: bytes and tokens summed, time = max
     (max_ms, max_e2e_ms), (all_bytes, all_tokens, all_e2e_bytes) = reduce_over_ranks(
@@ -339,7 +357,8 @@ def run_ours(args, w):
         dom = max(("dispatch", "combine"), key=lambda k: kern_ms[k])
         ach = abytes[dom] / (kern_ms[dom] * 1e-3) / 1e9
         kern_names = {"dispatch": "dispatch_fp8_kernel" if w.fp8 else "dispatch_bf16_kernel",
-                      "combine": "combine_kernel"}
+                      "combine": "combine_partial_kernel+combine_reduce_kernel" if two_level
+                      else "combine_kernel"}
         line = {
             "metric": METRIC, "value": round(all_bytes / (max_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -349,6 +368,7 @@ def run_ours(args, w):
             "tokens_per_s": round(all_tokens / (max_ms * 1e-3), 1),
             "config": config_of(w, extra={
                 "R_exp": R_exp, "R_disp": R_disp,
+                "combine": "two-level (per partition, then per token)" if two_level else "one-level",
                 "l2": "flushed between timed steps (256 MiB write + 256 MiB read, untimed)",
                 "timing": "one CUDA graph replay per step; CUDA events recorded inside the graph "
                           "on the launch stream bracket the step's kernels"}),
@@ -380,7 +400,8 @@ def run_ours(args, w):
     return 0
 
 
-def run_e2e(args, w, buf, idx_h, po_h, g_h, x, y, stream, dev, flush, step_bytes):
+def run_e2e(args, w, buf, idx_h, po_h, g_h, x, y, stream, dev, flush, step_bytes,
+            two_level=False):
     """Public-API calls on host inputs: pinned host -> device copies of every
     input, layout / dispatch / combine, device -> host copy of the output."""
     import torch
@@ -406,7 +427,7 @@ def run_e2e(args, w, buf, idx_h, po_h, g_h, x, y, stream, dev, flush, step_bytes
             s.record()
             for dst, src in ((d_idx, hidx), (d_po, hpo), (d_g, hg), (d_x, hx), (d_y, hy)):
                 dst.copy_(src, non_blocking=True)
-            out = buf.step(d_idx, d_po, d_x, d_y, d_g)
+            out = buf.step(d_idx, d_po, d_x, d_y, d_g, two_level=two_level)
             hout.copy_(out, non_blocking=True)
             e.record()
         e.synchronize()
@@ -445,6 +466,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(W.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--combine", choices=("one-level", "two-level"), default="one-level",
+                    help="two-level: per-partition reduce then per-token sum (dedup workloads)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3

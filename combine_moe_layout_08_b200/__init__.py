@@ -5,6 +5,8 @@ Python face of libmoe_layout.so, with the C names:
 * :func:`moe_layout`   -- routing layout (counts, prefix sums, row indices)
 * :func:`moe_dispatch` -- dispatch permute, optional dedup and FP8 e4m3 cast
 * :func:`moe_combine`  -- gate-weighted, slot-ordered combine
+* :func:`moe_combine_partial` / :func:`moe_combine_reduce` -- the two-level
+  combine of a deduplicated dispatch (per partition, then per token)
 
 Tensors are passed as device pointers with the current CUDA stream; this
 module checks dtypes, shapes and devices, allocates nothing inside the calls
@@ -26,7 +28,7 @@ from ._lib import (MOE_MAX_E_PART, MOE_MAX_G, MOE_MAX_TOPK, MOE_STATIC_SCRATCH_B
 
 __all__ = ["MoEProblem", "MoELayout", "MoEBuffers", "MoEError", "alloc_layout",
            "layout_workspace_size", "moe_layout", "moe_layout_static", "moe_dispatch",
-           "moe_combine",
+           "moe_combine", "moe_combine_partial", "moe_combine_reduce",
            "moe_status_string", "moe_abi_version", "MOE_STATUS_BAD_EXPERT",
            "MOE_STATUS_BAD_PART", "MOE_STATUS_BAD_ROW", "MOE_MAX_G", "MOE_MAX_E_PART",
            "MOE_MAX_TOPK"]
@@ -201,6 +203,41 @@ def moe_combine(prob: MoEProblem, y: torch.Tensor, topk_weights: torch.Tensor, l
         raise MoEError("moe_combine", rc)
 
 
+def moe_combine_partial(prob: MoEProblem, y: torch.Tensor, topk_weights: torch.Tensor,
+                        lay: MoELayout, z: torch.Tensor, stream=None) -> None:
+    """Partition side of the two-level (dedup) combine: z [M*topk, N] bf16 in
+    dispatch-row space, one row per (token, partition)."""
+    dev = y.device
+    if not prob.dedup:
+        raise ValueError("the two-level combine needs a dedup layout")
+    _check(y, "y", torch.bfloat16, prob.capacity * prob.N, dev)
+    _check(topk_weights, "topk_weights", torch.float32, prob.M * prob.topk, dev)
+    _check(z, "z", torch.bfloat16, prob.capacity * prob.N, dev)
+    _check_layout(prob, lay, dev)
+    s, l = prob.struct(), lay.struct()
+    rc = _lib.load().moe_combine_partial(ctypes.byref(s), y.data_ptr(), topk_weights.data_ptr(),
+                                         ctypes.byref(l), z.data_ptr(), _stream(y, stream))
+    if rc:
+        raise MoEError("moe_combine_partial", rc)
+
+
+def moe_combine_reduce(prob: MoEProblem, z: torch.Tensor, lay: MoELayout, out: torch.Tensor,
+                       stream=None) -> None:
+    """Token side of the two-level combine: out [M, N] bf16 = sum of the
+    token's partition rows of z, in partition order."""
+    dev = z.device
+    if not prob.dedup:
+        raise ValueError("the two-level combine needs a dedup layout")
+    _check(z, "z", torch.bfloat16, prob.capacity * prob.N, dev)
+    _check(out, "out", torch.bfloat16, prob.M * prob.N, dev)
+    _check_layout(prob, lay, dev)
+    s, l = prob.struct(), lay.struct()
+    rc = _lib.load().moe_combine_reduce(ctypes.byref(s), z.data_ptr(), ctypes.byref(l),
+                                        out.data_ptr(), _stream(z, stream))
+    if rc:
+        raise MoEError("moe_combine_reduce", rc)
+
+
 class MoEBuffers:
     """Caller-side device buffers of one problem at worst-case capacity, and
     the three calls of one pass over them (layout -> dispatch -> combine)."""
@@ -229,8 +266,20 @@ class MoEBuffers:
     def combine_(self, y, topk_weights, stream=None):
         moe_combine(self.prob, y, topk_weights, self.layout, self.out, stream)
 
-    def step(self, topk_idx, part_of, x, y, topk_weights, stream=None):
+    def combine_two_level_(self, y, topk_weights, stream=None):
+        """Two-level combine through the dispatch-row buffer ``self.z``
+        (allocated on first use)."""
+        if getattr(self, "z", None) is None:
+            self.z = torch.empty((max(self.prob.capacity, 1), self.prob.N), dtype=torch.bfloat16,
+                                 device=self.device)
+        moe_combine_partial(self.prob, y, topk_weights, self.layout, self.z, stream)
+        moe_combine_reduce(self.prob, self.z, self.layout, self.out, stream)
+
+    def step(self, topk_idx, part_of, x, y, topk_weights, stream=None, two_level=False):
         self.layout_(topk_idx, part_of, stream)
         self.dispatch_(x, stream)
-        self.combine_(y, topk_weights, stream)
+        if two_level:
+            self.combine_two_level_(y, topk_weights, stream)
+        else:
+            self.combine_(y, topk_weights, stream)
         return self.out

@@ -56,6 +56,12 @@ SIGNATURES = {
                                     ctypes.c_void_p]),
     "moe_combine": (ctypes.c_int, [ctypes.POINTER(ProblemStruct), ctypes.c_void_p, ctypes.c_void_p,
                                    ctypes.POINTER(LayoutStruct), ctypes.c_void_p, ctypes.c_void_p]),
+    "moe_combine_partial": (ctypes.c_int, [ctypes.POINTER(ProblemStruct), ctypes.c_void_p,
+                                           ctypes.c_void_p, ctypes.POINTER(LayoutStruct),
+                                           ctypes.c_void_p, ctypes.c_void_p]),
+    "moe_combine_reduce": (ctypes.c_int, [ctypes.POINTER(ProblemStruct), ctypes.c_void_p,
+                                          ctypes.POINTER(LayoutStruct), ctypes.c_void_p,
+                                          ctypes.c_void_p]),
 }
 
 _lock = threading.Lock()

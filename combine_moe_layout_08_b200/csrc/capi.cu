@@ -91,4 +91,25 @@ int moe_combine(const moe_problem_t* prob, const void* y, const float* topk_weig
                                      reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int moe_combine_partial(const moe_problem_t* prob, const void* y, const float* topk_weights,
+                        const moe_layout_t* lay, void* z, moe_stream_t stream) {
+  if (!valid_problem(prob) || !valid_layout(prob, lay) || !prob->dedup) return MOE_ERR_ARG;
+  if (prob->M > 0) {
+    if (!y || !aligned(y, 16) || !z || !aligned(z, 16)) return MOE_ERR_ARG;
+    if (!arr(topk_weights)) return MOE_ERR_ARG;
+  }
+  return cuda_rc(moe::launch_combine_partial(*prob, y, topk_weights, *lay, z,
+                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int moe_combine_reduce(const moe_problem_t* prob, const void* z, const moe_layout_t* lay,
+                       void* out, moe_stream_t stream) {
+  if (!valid_problem(prob) || !valid_layout(prob, lay) || !prob->dedup) return MOE_ERR_ARG;
+  if (prob->M > 0) {
+    if (!z || !aligned(z, 16) || !out || !aligned(out, 16)) return MOE_ERR_ARG;
+  }
+  return cuda_rc(moe::launch_combine_reduce(*prob, z, *lay, out,
+                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

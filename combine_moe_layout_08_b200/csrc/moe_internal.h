@@ -59,6 +59,12 @@ cudaError_t launch_dispatch(const moe_problem_t& p, const void* x,
                             const moe_layout_t& lay, void* recv_x,
                             float* recv_scale, cudaStream_t stream);
 
+cudaError_t launch_combine_partial(const moe_problem_t& p, const void* y, const float* w,
+                                   const moe_layout_t& lay, void* z, cudaStream_t stream);
+
+cudaError_t launch_combine_reduce(const moe_problem_t& p, const void* z, const moe_layout_t& lay,
+                                  void* out, cudaStream_t stream);
+
 cudaError_t launch_combine(const moe_problem_t& p, const void* y,
                            const float* w, const moe_layout_t& lay, void* out,
                            cudaStream_t stream);

@@ -208,6 +208,40 @@ int moe_combine(const moe_problem_t *prob, const void *y,
                 const float *topk_weights, const moe_layout_t *lay, void *out,
                 moe_stream_t stream);
 
+/*
+ * Two-level combine of a deduplicated dispatch (prob->dedup = 1, else
+ * MOE_ERR_ARG): the return path of per-partition dedup, where each
+ * partition first reduces the outputs of a token's experts it holds and the
+ * token then sums its partitions (Zyphra news item, correlated expert
+ * placement: one copy of a token per GPU each way; Purlin section 3.3,
+ * SCORE: one owner per output element, source-order accumulation).
+ * Results differ from moe_combine by the extra bf16 rounding of each
+ * partition's partial sum.
+ *
+ * moe_combine_partial -- partition side:
+ *   z[disp_row[t,p], :] = bf16( sum over slots k of t whose expert is on
+ *                         partition p, in slot order, of w[t,k] *
+ *                         y[exp_row[t,k], :] )   (fp32 fma from +0)
+ *   y             [M*topk, N] bf16 expert outputs in expert-row space
+ *   topk_weights  [M, topk] fp32
+ *   z             [M*topk, N] bf16 in dispatch-row space; rows [0, R_disp)
+ *                 are written (the payload that returns to the tokens)
+ * moe_combine_reduce -- token side:
+ *   out[t, :] = bf16( sum over p = 0..E_part-1 with disp_row[t,p] >= 0 of
+ *               z[disp_row[t,p], :] )   (fp32 additions from +0)
+ *   out           [M, N] bf16
+ * Both are asynchronous on `stream`; run moe_combine_partial before
+ * moe_combine_reduce on one stream (or order them with an event).  z is the
+ * caller's buffer, 16-byte aligned like y and out.  Row indices outside
+ * [0, M*topk) in exp_row, exp_to_disp or disp_row are skipped and raise
+ * MOE_STATUS_BAD_ROW in lay->status; the calls never trap.
+ */
+int moe_combine_partial(const moe_problem_t *prob, const void *y,
+                        const float *topk_weights, const moe_layout_t *lay,
+                        void *z, moe_stream_t stream);
+int moe_combine_reduce(const moe_problem_t *prob, const void *z,
+                       const moe_layout_t *lay, void *out, moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

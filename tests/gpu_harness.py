@@ -128,3 +128,32 @@ def compare_combine(b: moe.MoEBuffers, prob, y_dev, weights, exp_row, tokens=Non
     d = ulp_distance_bf16(got, want)
     assert d.max(initial=0) <= max_ulp, f"combine differs by {d.max()} bf16 steps"
     return int(np.count_nonzero(got != want))
+
+
+def compare_two_level(b: moe.MoEBuffers, prob, y_dev, gates, idx, part_of, ref, tokens=None,
+                      max_ulp=1):
+    """Two-level combine: the partition rows z (all, or those of the sample
+    ``tokens``) bit-exact, and out within max_ulp bf16 steps of the oracle
+    (which runs on a compact copy of the sampled tokens); returns the number
+    of out elements that differ at all."""
+    M, topk = idx.shape
+    E = prob.E_part
+    tok = np.arange(M) if tokens is None else np.asarray(tokens, np.int64)
+    n = tok.size
+    er = ref["exp_row"][tok]
+    dr = ref["disp_row"][tok]
+    valid = er >= 0
+    rows = np.where(valid, er, 0).ravel()
+    y_sub = oracle.bf16_bits(y_dev[torch.from_numpy(rows).to(y_dev.device)])
+    er_sub = np.where(valid, np.arange(n * topk).reshape(n, topk), -1).astype(np.int32)
+    dvalid = dr >= 0
+    dr_sub = np.where(dvalid, np.arange(n * E).reshape(n, E), -1).astype(np.int32)
+    lay_sub = dict(exp_row=er_sub, disp_row=dr_sub, R_disp=n * E)
+    z_ref = oracle.combine_partial(y_sub, gates[tok], idx[tok], part_of, lay_sub)
+    out_ref = oracle.combine_reduce(z_ref, dr_sub)
+    z_got = oracle.bf16_bits(b.z[torch.from_numpy(dr[dvalid].astype(np.int64)).to(b.z.device)])
+    np.testing.assert_array_equal(z_got, z_ref[dr_sub[dvalid]])
+    got = oracle.bf16_bits(b.out[torch.from_numpy(tok).to(b.out.device)])
+    d = ulp_distance_bf16(got, out_ref)
+    assert d.max(initial=0) <= max_ulp, f"two-level combine differs by {d.max()} bf16 steps"
+    return int(np.count_nonzero(got != out_ref))

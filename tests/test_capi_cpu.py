@@ -129,6 +129,12 @@ def test_dispatch_combine_reject_bad_arguments(L):
     assert L.moe_combine(p, FAKE, FAKE + 2, ctypes.byref(lay), FAKE, None) == 1
     assert L.moe_combine(p, FAKE, FAKE, ctypes.byref(lay), FAKE + 8, None) == 1
     assert L.moe_combine(ctypes.byref(P(N=0)), FAKE, FAKE, ctypes.byref(lay), FAKE, None) == 1
+    # the two-level combine needs a dedup problem
+    assert L.moe_combine_partial(p, FAKE, FAKE, ctypes.byref(lay), FAKE, None) == 1
+    assert L.moe_combine_reduce(p, FAKE, ctypes.byref(lay), FAKE, None) == 1
+    pd = ctypes.byref(P(dedup=1))
+    assert L.moe_combine_partial(pd, FAKE + 4, FAKE, ctypes.byref(lay), FAKE, None) == 1
+    assert L.moe_combine_reduce(pd, FAKE, ctypes.byref(lay), FAKE + 8, None) == 1
 
 
 def test_python_binding_fails_loudly_without_library(monkeypatch, tmp_path):
