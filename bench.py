@@ -248,6 +248,27 @@ def config_of(w, extra=None):
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
+def graph_kernel_nodes(graph) -> int:
+    """Kernel nodes of a captured (not yet instantiated) step graph: the
+    launches of this library's kernels per step (the graph holds nothing
+    else but event records)."""
+    from cuda.bindings import runtime as rt
+    raw = graph.raw_cuda_graph()
+    err, _, n = rt.cudaGraphGetNodes(raw, 0)
+    if err != rt.cudaError_t.cudaSuccess:
+        raise RuntimeError(f"cudaGraphGetNodes: {err}")
+    err, nodes, n = rt.cudaGraphGetNodes(raw, n)
+    if err != rt.cudaError_t.cudaSuccess:
+        raise RuntimeError(f"cudaGraphGetNodes: {err}")
+    kernels = 0
+    for node in nodes[:n]:
+        err, kind = rt.cudaGraphNodeGetType(node)
+        if err != rt.cudaError_t.cudaSuccess:
+            raise RuntimeError(f"cudaGraphNodeGetType: {err}")
+        kernels += kind == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel
+    return kernels
+
+
 def run_ours(args, w):
     import torch
     import torch.distributed as dist
@@ -282,31 +303,48 @@ def run_ours(args, w):
         flush_w.zero_()
         torch.sum(flush_r, dim=0, out=flush_sink)
 
+    two_level = args.combine == "two-level"
+    if two_level and not w.dedup:
+        raise SystemExit("--combine two-level needs a dedup workload")
+    separate = args.schedule == "separate"
+    fused = not separate and moe.moe_layout_dispatch_fused(prob)
     # eager warm-up through the public API, then one graph per step with
     # external events between the kernels
     with torch.cuda.stream(stream):
         for _ in range(3):
-            buf.step(idx, po, x, y, gates, two_level=args.combine == "two-level")
+            buf.step(idx, po, x, y, gates, two_level=two_level, separate=separate)
     stream.synchronize()
-    two_level = args.combine == "two-level"
-    if two_level and not w.dedup:
-        raise SystemExit("--combine two-level needs a dedup workload")
-    # events inside the graph bracket the step's kernels on the device (the
-    # graph's own launch latency, which back-to-back steps hide, stays out)
-    names = ["layout", "dispatch"] + (["combine_partial", "combine_reduce"] if two_level else ["combine"])
-    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(names) + 1)]
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        ev[0].record()
-        buf.layout_(idx, po)
-        ev[1].record()
-        buf.dispatch_(x)
-        ev[2].record()
-        if two_level:
-            buf.combine_two_level_(y, gates)  # two kernels: events only around the pair
-        else:
-            buf.combine_(y, gates)
-        ev[3].record()
+    # Two graphs of the same step.  The timed one has events only at its two
+    # ends, so consecutive kernels keep their programmatic (early-launch)
+    # edges as in production; the second has events between the kernels for
+    # the per-kernel breakdown (an event node between two kernels replaces
+    # that edge with a full dependency, so its parts add up to a little more
+    # than the step).
+    def capture(inner):
+        ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+        mark = (lambda i: ev[i].record()) if inner else (lambda i: None)
+        graph = torch.cuda.CUDAGraph(keep_graph=True)
+        with torch.cuda.graph(graph, stream=stream):
+            ev[0].record()
+            if fused:  # one kernel: layout and dispatch share one interval
+                buf.layout_dispatch_(idx, po, x)
+                mark(1)
+            else:
+                buf.layout_(idx, po)
+                mark(1)
+                buf.dispatch_(x)
+            mark(2)
+            if two_level:
+                buf.combine_two_level_(y, gates)  # two kernels: events only around the pair
+            else:
+                buf.combine_(y, gates)
+            ev[3].record()
+        n = graph_kernel_nodes(graph)
+        graph.instantiate()
+        return graph, ev, n
+
+    graph, ev, launches_per_step = capture(inner=False)
+    pgraph, pev, _ = capture(inner=True)
     R_exp = int(buf.layout.expert_offset[w.G].item())
     R_disp = int(buf.layout.part_offset[w.E_part].item())
     status = int(buf.layout.status.item())
@@ -316,36 +354,53 @@ def run_ours(args, w):
     if two_level:  # one timed interval covers both combine kernels
         abytes = {"layout": abytes["layout"], "dispatch": abytes["dispatch"],
                   "combine": abytes["combine_partial"] + abytes["combine_reduce"]}
+    if fused:
+        abytes = {"layout+dispatch": abytes["layout"] + abytes["dispatch"],
+                  "combine": abytes["combine"]}
     step_bytes = sum(abytes.values())
+    move = "layout+dispatch" if fused else "dispatch"
 
     def timed_step():
         with torch.cuda.stream(stream):
             flush()
             graph.replay()
         stream.synchronize()
-        return (ev[0].elapsed_time(ev[3]), ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2]),
-                ev[2].elapsed_time(ev[3]))
+        return ev[0].elapsed_time(ev[3])
+
+    def parts_step():
+        with torch.cuda.stream(stream):
+            flush()
+            pgraph.replay()
+        stream.synchronize()
+        return (pev[0].elapsed_time(pev[3]), pev[0].elapsed_time(pev[1]),
+                pev[1].elapsed_time(pev[2]), pev[2].elapsed_time(pev[3]))
 
     for _ in range(max(args.warmup, 3)):
         timed_step()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    per = []
+    step_ms = []
     with ClockSampler(dev) as clk:
         for _ in range(args.steps):
-            per.append(timed_step())
+            step_ms.append(timed_step())
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
-    per = np.array(per)                                 # [K, 4] ms
-    total_ms = float(per[:, 0].sum())
-    kern_ms = {"layout": float(per[:, 1].mean()), "dispatch": float(per[:, 2].mean()),
-               "combine": float(per[:, 3].mean())}
+    total_ms = float(np.sum(step_ms))
+    # per-kernel breakdown (untimed for the headline; same flush, same inputs)
+    for _ in range(3):
+        parts_step()
+    per = np.array([parts_step() for _ in range(args.steps)])   # [K, 4] ms
+    if fused:
+        kern_ms = {"layout+dispatch": float(per[:, 1].mean()), "combine": float(per[:, 3].mean())}
+    else:
+        kern_ms = {"layout": float(per[:, 1].mean()), "dispatch": float(per[:, 2].mean()),
+                   "combine": float(per[:, 3].mean())}
 
     # end to end through the public API with host buffers
     e2e = run_e2e(args, wr, buf, idx_h, po_h, g_h, x, y, stream, dev, flush, step_bytes,
-                  two_level)
+                  two_level, separate)
 
     # aggregate over ranks: bytes and tokens summed, time = max
     (max_ms, max_e2e_ms), (all_bytes, all_tokens, all_e2e_bytes) = reduce_over_ranks(
@@ -354,9 +409,10 @@ def run_ours(args, w):
     line = None
     if rank == 0:
         peak, peak_kind = measured_peak()
-        dom = max(("dispatch", "combine"), key=lambda k: kern_ms[k])
+        dom = max((move, "combine"), key=lambda k: kern_ms[k])
         ach = abytes[dom] / (kern_ms[dom] * 1e-3) / 1e9
         kern_names = {"dispatch": "dispatch_fp8_kernel" if w.fp8 else "dispatch_bf16_kernel",
+                      "layout+dispatch": "layout_dispatch_kernel",
                       "combine": "combine_partial_kernel+combine_reduce_kernel" if two_level
                       else "combine_kernel"}
         line = {
@@ -369,10 +425,14 @@ def run_ours(args, w):
             "config": config_of(w, extra={
                 "R_exp": R_exp, "R_disp": R_disp,
                 "combine": "two-level (per partition, then per token)" if two_level else "one-level",
+                "schedule": "one kernel for layout + dispatch" if fused else
+                            "separate layout and dispatch kernels",
                 "l2": "flushed between timed steps (256 MiB write + 256 MiB read, untimed)",
                 "timing": "one CUDA graph replay per step; CUDA events recorded inside the graph "
-                          "on the launch stream bracket the step's kernels"}),
+                          "on the launch stream at its start and end"}),
             "kernels_us": {k: round(v * 1e3, 2) for k, v in kern_ms.items()},
+            "kernels_note": "per-kernel times from a second graph of the step with events "
+                            "between its kernels (mean over the same number of steps)",
             "kernels_gbs": {k: round(abytes[k] / (kern_ms[k] * 1e-3) / 1e9, 1) for k in kern_ms},
             "algorithmic_bytes_per_step": abytes,
             "roofline": {"bound": "hbm", "kernel": kern_names[dom], "achieved": round(ach, 1),
@@ -380,16 +440,17 @@ def run_ours(args, w):
                          "peak_kind": f"of {peak_kind}",
                          "traffic": traffic_record(kern_names[dom], w.name)},
             "frac_of_8tbs": {k: round(abytes[k] / (kern_ms[k] * 1e-3) / 8e12, 4) for k in
-                             ("dispatch", "combine")},
+                             (move, "combine")},
             "e2e": {"value": round(all_e2e_bytes / (max_e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                     "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                     "tokens_per_s": round(w.M * world * args.steps / (max_e2e_ms * 1e-3), 1),
                     "ms_per_step": round(max_e2e_ms / args.steps, 4),
                     "steps": e2e["steps"]},
-            "gpu_launches": 4 * args.steps,
+            "gpu_launches": launches_per_step * args.steps,
             "clocks": clk.summary(),
         }
     graph.reset()
+    pgraph.reset()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -401,7 +462,7 @@ def run_ours(args, w):
 
 
 def run_e2e(args, w, buf, idx_h, po_h, g_h, x, y, stream, dev, flush, step_bytes,
-            two_level=False):
+            two_level=False, separate=False):
     """Public-API calls on host inputs: pinned host -> device copies of every
     input, layout / dispatch / combine, device -> host copy of the output."""
     import torch
@@ -427,7 +488,7 @@ def run_e2e(args, w, buf, idx_h, po_h, g_h, x, y, stream, dev, flush, step_bytes
             s.record()
             for dst, src in ((d_idx, hidx), (d_po, hpo), (d_g, hg), (d_x, hx), (d_y, hy)):
                 dst.copy_(src, non_blocking=True)
-            out = buf.step(d_idx, d_po, d_x, d_y, d_g, two_level=two_level)
+            out = buf.step(d_idx, d_po, d_x, d_y, d_g, two_level=two_level, separate=separate)
             hout.copy_(out, non_blocking=True)
             e.record()
         e.synchronize()
@@ -458,6 +519,81 @@ def cpu_baseline(w, buf, idx_h, po_h, g_h, x, y, budget_s=10.0):
                       f"{sum(times):.1f} s, single thread"}
 
 
+def run_latency_sweep(args):
+    """Decode latency against M on one GPU, in the shape of the Triton-
+    distributed issue #117 table (N = 7168, G = 256, topk = 8, bf16,
+    M = 2..512): median device time of layout + dispatch (one call, and the
+    separate calls) and of combine, L2 flushed before each step.  Prints one
+    JSON line; context for the decode path, not the contract line.  Event
+    timestamps on this part advance in steps of about 2 us, so single
+    intervals of a few us are coarse; medians over many steps are reported.
+    step_us comes from a graph with events only at its ends; the parts from
+    a graph with an event between them."""
+    import dataclasses
+
+    import torch
+
+    import combine_moe_layout_08_b200 as moe
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    base = W.get("decode-M128-uniform")
+    stream = torch.cuda.Stream(dev)
+    flush_w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    rows = []
+    for M in (2, 4, 8, 16, 32, 64, 128, 256, 512):
+        w = dataclasses.replace(base, name=f"decode-M{M}-uniform", M=M)
+        d = W.make_inputs(w, device=dev)
+        prob = moe.MoEProblem(w.M, w.N, w.G, w.topk, w.E_part, w.dedup, w.fp8)
+        idx = torch.from_numpy(d["topk_idx"]).to(dev)
+        po = torch.from_numpy(d["part_of"]).to(dev)
+        gates = torch.from_numpy(d["topk_weights"]).to(dev)
+        row = {"M": M, "one_kernel": moe.moe_layout_dispatch_fused(prob)}
+        for separate in (False, True):
+            buf = moe.MoEBuffers(prob, dev)
+            with torch.cuda.stream(stream):
+                buf.step(idx, po, d["x"], d["y"], gates, separate=separate)
+            stream.synchronize()
+            med = []
+            for inner in (False, True):  # the whole step, then its two parts
+                ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
+                graph = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(graph, stream=stream):
+                    ev[0].record()
+                    if separate:
+                        buf.layout_(idx, po)
+                        buf.dispatch_(d["x"])
+                    else:
+                        buf.layout_dispatch_(idx, po, d["x"])
+                    if inner:
+                        ev[1].record()
+                    buf.combine_(d["y"], gates)
+                    ev[2].record()
+                t = []
+                for i in range(max(args.warmup, 3) + args.steps):
+                    with torch.cuda.stream(stream):
+                        flush_w.zero_()
+                        graph.replay()
+                    stream.synchronize()
+                    if i >= max(args.warmup, 3):
+                        t.append((ev[0].elapsed_time(ev[2]),) + ((ev[0].elapsed_time(ev[1]),
+                                                                  ev[1].elapsed_time(ev[2]))
+                                                                 if inner else (0.0, 0.0)))
+                med.append(np.median(np.array(t), axis=0) * 1e3)
+                graph.reset()
+            key = "separate_" if separate else ""
+            row[key + "step_us"] = round(float(med[0][0]), 2)
+            row[key + "layout_dispatch_us"] = round(float(med[1][1]), 2)
+            if not separate:
+                row["combine_us"] = round(float(med[1][2]), 2)
+        rows.append(row)
+    print(json.dumps({"metric": "decode latency against M (us, median, L2 flushed)",
+                      "config": {"N": base.N, "G": base.G, "topk": base.topk,
+                                 "E_part": base.E_part, "routing": base.routing},
+                      "steps": args.steps, "rows": rows}), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -466,11 +602,17 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(W.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--schedule", choices=("auto", "separate"), default="auto",
+                    help="separate: moe_layout + moe_dispatch even where one kernel does both")
     ap.add_argument("--combine", choices=("one-level", "two-level"), default="one-level",
                     help="two-level: per-partition reduce then per-token sum (dedup workloads)")
+    ap.add_argument("--latency-sweep", action="store_true",
+                    help="decode latency for M = 2..512 (one JSON line; not the contract line)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
+    if args.latency_sweep:
+        return run_latency_sweep(args)
     w = W.get(args.workload)
     if args.impl == "reference":
         return run_reference(args, w)

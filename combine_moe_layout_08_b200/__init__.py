@@ -28,7 +28,7 @@ from ._lib import (MOE_MAX_E_PART, MOE_MAX_G, MOE_MAX_TOPK, MOE_STATIC_SCRATCH_B
 
 __all__ = ["MoEProblem", "MoELayout", "MoEBuffers", "MoEError", "alloc_layout",
            "layout_workspace_size", "moe_layout", "moe_layout_static", "moe_dispatch",
-           "moe_combine", "moe_combine_partial", "moe_combine_reduce",
+           "moe_layout_dispatch", "moe_layout_dispatch_fused", "moe_combine", "moe_combine_partial", "moe_combine_reduce",
            "moe_status_string", "moe_abi_version", "MOE_STATUS_BAD_EXPERT",
            "MOE_STATUS_BAD_PART", "MOE_STATUS_BAD_ROW", "MOE_MAX_G", "MOE_MAX_E_PART",
            "MOE_MAX_TOPK"]
@@ -188,6 +188,37 @@ def moe_dispatch(prob: MoEProblem, x: torch.Tensor, lay: MoELayout, recv_x: torc
         raise MoEError("moe_dispatch", rc)
 
 
+def moe_layout_dispatch(prob: MoEProblem, topk_idx: torch.Tensor, part_of: torch.Tensor,
+                        lay: MoELayout, workspace: torch.Tensor, x: torch.Tensor,
+                        recv_x: torch.Tensor, recv_scale: Optional[torch.Tensor] = None,
+                        stream=None) -> None:
+    """moe_layout then moe_dispatch in one call (bit-identical results); small
+    batches run as one kernel (see ``moe_layout_dispatch_fused``)."""
+    dev = x.device
+    cap = prob.capacity
+    _check(topk_idx, "topk_idx", torch.int32, prob.M * prob.topk, dev)
+    _check(part_of, "part_of", torch.int32, prob.G, dev)
+    _check(workspace, "workspace", torch.uint8, None, dev)
+    _check(x, "x", torch.bfloat16, prob.M * prob.N, dev)
+    _check(recv_x, "recv_x", torch.uint8 if prob.fp8 else torch.bfloat16, cap * prob.N, dev)
+    if prob.fp8:
+        _check(recv_scale, "recv_scale", torch.float32, cap * (prob.N // 128), dev)
+    _check_layout(prob, lay, dev)
+    s, l = prob.struct(), lay.struct()
+    rc = _lib.load().moe_layout_dispatch(
+        ctypes.byref(s), topk_idx.data_ptr(), part_of.data_ptr(), ctypes.byref(l),
+        workspace.data_ptr(), workspace.numel(), x.data_ptr(), recv_x.data_ptr(),
+        recv_scale.data_ptr() if recv_scale is not None else None, _stream(x, stream))
+    if rc:
+        raise MoEError("moe_layout_dispatch", rc)
+
+
+def moe_layout_dispatch_fused(prob: MoEProblem) -> bool:
+    """True if moe_layout_dispatch runs ``prob`` as one kernel."""
+    s = prob.struct()
+    return bool(_lib.load().moe_layout_dispatch_fused(ctypes.byref(s)))
+
+
 def moe_combine(prob: MoEProblem, y: torch.Tensor, topk_weights: torch.Tensor, lay: MoELayout,
                 out: torch.Tensor, stream=None) -> None:
     """out [M, N] bf16 = gate-weighted sum of the expert rows ``y`` [M*topk, N] bf16."""
@@ -263,6 +294,10 @@ class MoEBuffers:
     def dispatch_(self, x, stream=None):
         moe_dispatch(self.prob, x, self.layout, self.recv_x, self.recv_scale, stream)
 
+    def layout_dispatch_(self, topk_idx, part_of, x, stream=None):
+        moe_layout_dispatch(self.prob, topk_idx, part_of, self.layout, self.workspace, x,
+                            self.recv_x, self.recv_scale, stream)
+
     def combine_(self, y, topk_weights, stream=None):
         moe_combine(self.prob, y, topk_weights, self.layout, self.out, stream)
 
@@ -275,9 +310,15 @@ class MoEBuffers:
         moe_combine_partial(self.prob, y, topk_weights, self.layout, self.z, stream)
         moe_combine_reduce(self.prob, self.z, self.layout, self.out, stream)
 
-    def step(self, topk_idx, part_of, x, y, topk_weights, stream=None, two_level=False):
-        self.layout_(topk_idx, part_of, stream)
-        self.dispatch_(x, stream)
+    def step(self, topk_idx, part_of, x, y, topk_weights, stream=None, two_level=False,
+             separate=False):
+        """layout -> dispatch -> combine; ``separate`` calls moe_layout and
+        moe_dispatch instead of moe_layout_dispatch (same results)."""
+        if separate:
+            self.layout_(topk_idx, part_of, stream)
+            self.dispatch_(x, stream)
+        else:
+            self.layout_dispatch_(topk_idx, part_of, x, stream)
         if two_level:
             self.combine_two_level_(y, topk_weights, stream)
         else:

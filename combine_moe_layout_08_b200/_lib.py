@@ -54,6 +54,11 @@ SIGNATURES = {
     "moe_dispatch": (ctypes.c_int, [ctypes.POINTER(ProblemStruct), ctypes.c_void_p,
                                     ctypes.POINTER(LayoutStruct), ctypes.c_void_p, ctypes.c_void_p,
                                     ctypes.c_void_p]),
+    "moe_layout_dispatch": (ctypes.c_int, [ctypes.POINTER(ProblemStruct), ctypes.c_void_p,
+                                           ctypes.c_void_p, ctypes.POINTER(LayoutStruct),
+                                           ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
+                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "moe_layout_dispatch_fused": (ctypes.c_int, [ctypes.POINTER(ProblemStruct)]),
     "moe_combine": (ctypes.c_int, [ctypes.POINTER(ProblemStruct), ctypes.c_void_p, ctypes.c_void_p,
                                    ctypes.POINTER(LayoutStruct), ctypes.c_void_p, ctypes.c_void_p]),
     "moe_combine_partial": (ctypes.c_int, [ctypes.POINTER(ProblemStruct), ctypes.c_void_p,

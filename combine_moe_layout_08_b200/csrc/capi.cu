@@ -80,6 +80,31 @@ int moe_dispatch(const moe_problem_t* prob, const void* x, const moe_layout_t* l
                                       reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int moe_layout_dispatch_fused(const moe_problem_t* prob) {
+  return valid_problem(prob) && moe::layout_dispatch_fused(*prob) ? 1 : 0;
+}
+
+int moe_layout_dispatch(const moe_problem_t* prob, const int32_t* topk_idx,
+                        const int32_t* part_of, const moe_layout_t* lay, void* workspace,
+                        size_t workspace_bytes, const void* x, void* recv_x, float* recv_scale,
+                        moe_stream_t stream) {
+  if (!valid_problem(prob) || !valid_layout(prob, lay)) return MOE_ERR_ARG;
+  if (!arr(part_of) || (prob->M > 0 && !arr(topk_idx))) return MOE_ERR_ARG;
+  if (prob->M > 0) {
+    if (!x || !aligned(x, 16) || !recv_x || !aligned(recv_x, 16)) return MOE_ERR_ARG;
+    if (prob->fp8 && (!recv_scale || !aligned(recv_scale, 16))) return MOE_ERR_ARG;
+  }
+  const size_t need = moe::layout_workspace_bytes(*prob);
+  if (!workspace || !aligned(workspace, 16) || workspace_bytes < need) return MOE_ERR_WORKSPACE;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (moe::layout_dispatch_fused(*prob))
+    return cuda_rc(moe::launch_layout_dispatch(*prob, topk_idx, part_of, *lay, x, recv_x,
+                                               recv_scale, s));
+  cudaError_t e = moe::launch_layout(*prob, topk_idx, part_of, *lay, workspace, s);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  return cuda_rc(moe::launch_dispatch(*prob, x, *lay, recv_x, recv_scale, s));
+}
+
 int moe_combine(const moe_problem_t* prob, const void* y, const float* topk_weights,
                 const moe_layout_t* lay, void* out, moe_stream_t stream) {
   if (!valid_problem(prob) || !valid_layout(prob, lay)) return MOE_ERR_ARG;

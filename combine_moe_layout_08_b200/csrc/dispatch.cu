@@ -14,10 +14,9 @@
 // saturating round-to-nearest-even conversion; the 16 bytes of a lane are
 // stored to every destination and one lane of the 8 writes the block's
 // scale.  The quantisation is done once per token, not once per copy.
-#include <cuda_fp8.h>
-
 #include <algorithm>
 
+#include "fp8_device.cuh"
 #include "moe_device.cuh"
 #include "moe_internal.h"
 
@@ -113,34 +112,6 @@ __global__ void __launch_bounds__(kDThreads, 8) dispatch_bf16_kernel(DispatchArg
   }
 }
 
-// 16 bf16 values (two 16-byte chunks) -> 16 e4m3 bytes, given the block scale
-__device__ __forceinline__ uint4 quantize16(const uint4& lo, const uint4& hi, float scale) {
-  const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-  uint32_t q[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 f0 = make_float2(__fdiv_rn(bf16_lo(w[2 * i]), scale), __fdiv_rn(bf16_hi(w[2 * i]), scale));
-    const float2 f1 =
-        make_float2(__fdiv_rn(bf16_lo(w[2 * i + 1]), scale), __fdiv_rn(bf16_hi(w[2 * i + 1]), scale));
-    const uint32_t b0 = __nv_cvt_float2_to_fp8x2(f0, __NV_SATFINITE, __NV_E4M3);
-    const uint32_t b1 = __nv_cvt_float2_to_fp8x2(f1, __NV_SATFINITE, __NV_E4M3);
-    q[i] = (b0 & 0xffffu) | (b1 << 16);
-  }
-  return make_uint4(q[0], q[1], q[2], q[3]);
-}
-
-__device__ __forceinline__ float absmax8(const uint4& v) {
-  float m = fabsf(bf16_lo(v.x));
-  m = fmaxf(m, fabsf(bf16_hi(v.x)));
-  m = fmaxf(m, fabsf(bf16_lo(v.y)));
-  m = fmaxf(m, fabsf(bf16_hi(v.y)));
-  m = fmaxf(m, fabsf(bf16_lo(v.z)));
-  m = fmaxf(m, fabsf(bf16_hi(v.z)));
-  m = fmaxf(m, fabsf(bf16_lo(v.w)));
-  m = fmaxf(m, fabsf(bf16_hi(v.w)));
-  return m;
-}
-
 // Each thread owns a 16-column group g; 8 consecutive lanes form one
 // 128-column scale block.  N is a multiple of 128 and kDThreads of 8, so a
 // lane group is either entirely inside the row or entirely past its end.
@@ -171,19 +142,7 @@ __global__ void __launch_bounds__(kDThreads, 8) dispatch_fp8_kernel(DispatchArgs
   uint4 q[U];
   float s[U];
 #pragma unroll
-  for (int u = 0; u < U; ++u) {
-    float m = fmaxf(absmax8(lo[u]), absmax8(hi[u]));
-    m = fmaxf(m, __shfl_xor_sync(kFull, m, 1));
-    m = fmaxf(m, __shfl_xor_sync(kFull, m, 2));
-    m = fmaxf(m, __shfl_xor_sync(kFull, m, 4));
-    if (m == 0.0f) {
-      s[u] = 0.0f;
-      q[u] = make_uint4(0, 0, 0, 0);
-    } else {
-      s[u] = __fdiv_rn(m, 448.0f);
-      q[u] = quantize16(lo[u], hi[u], s[u]);
-    }
-  }
+  for (int u = 0; u < U; ++u) q[u] = quantize_lane(lo[u], hi[u], s[u]);
   uint4* recv = static_cast<uint4*>(a.recv);  // a row is N bytes = N16 chunks
   const int N128 = N16 >> 3;
   const bool scale_lane = (threadIdx.x & 7) == 0;

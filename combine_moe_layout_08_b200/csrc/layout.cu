@@ -38,6 +38,7 @@
 
 #include <algorithm>
 
+#include "layout_device.cuh"
 #include "moe_device.cuh"
 #include "moe_internal.h"
 
@@ -97,8 +98,6 @@ struct LayoutArgs {
   int* exp_to_disp;
   int* status;
 };
-
-__device__ __forceinline__ bool valid_part(int p, int E) { return p >= 0 && p < E; }
 
 struct Tile {
   int t0, ntok, n_items;
@@ -270,56 +269,10 @@ __device__ void rank_assign(int n, int K, int* whist, KeyOf key_of, OnRank on_ra
   __syncthreads();
 }
 
-// One warp: in-place exclusive scan of data[0..n); returns the total.
-__device__ int warp_exclusive_scan(int* data, int n) {
-  const int lane = lane_id();
-  const int per = (n + kWarp - 1) / kWarp;
-  const int beg = min(n, lane * per), end = min(n, beg + per);
-  int s = 0;
-  for (int i = beg; i < end; ++i) s += data[i];
-  int x = s;
-#pragma unroll
-  for (int o = 1; o < kWarp; o <<= 1) {
-    const int y = __shfl_up_sync(kFull, x, o);
-    if (lane >= o) x += y;
-  }
-  int run = x - s;
-  for (int i = beg; i < end; ++i) {
-    const int v = data[i];
-    data[i] = run;
-    run += v;
-  }
-  return __shfl_sync(kFull, x, kWarp - 1);
-}
-
 // One warp: position of every expert in (partition, id) order, experts with
 // an invalid placement last.  Reads only the placement map.
-__device__ void expert_order(const LayoutArgs& a, const Smem& S) {
-  const int lane = lane_id(), G = a.G, E = a.E;
-  for (int k = lane; k <= E; k += kWarp) S.kcnt[k] = 0;
-  __syncwarp();
-  const int nbits = key_bits(E + 1);
-  const unsigned lt = lanemask_lt();
-  for (int c = 0; c < G; c += kWarp) {
-    const int e = c + lane;
-    int key = -1;
-    if (e < G) key = valid_part(S.part_s[e], E) ? S.part_s[e] : E;
-    const unsigned peers = match_peers(key, nbits);
-    const int base = key >= 0 ? S.kcnt[key] : 0;
-    __syncwarp();
-    if (key >= 0) {
-      S.pos[e] = base + __popc(peers & lt);  // rank among the experts of its key
-      if (lane == __ffs(peers) - 1) S.kcnt[key] = base + __popc(peers);
-    }
-    __syncwarp();
-  }
-  (void)warp_exclusive_scan(S.kcnt, E + 1);  // start of each key
-  __syncwarp();
-  for (int e = lane; e < G; e += kWarp) {
-    const int key = valid_part(S.part_s[e], E) ? S.part_s[e] : E;
-    S.pos[e] += S.kcnt[key];
-  }
-  __syncwarp();
+__device__ __forceinline__ void expert_order(const LayoutArgs& a, const Smem& S) {
+  expert_order_warp(S.part_s, a.G, a.E, S.pos, S.kcnt);
 }
 
 // Partition bit mask of token tl of the tile (valid pairs only).

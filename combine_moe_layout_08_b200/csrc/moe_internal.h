@@ -59,6 +59,13 @@ cudaError_t launch_dispatch(const moe_problem_t& p, const void* x,
                             const moe_layout_t& lay, void* recv_x,
                             float* recv_scale, cudaStream_t stream);
 
+// One-kernel layout + dispatch: taken for 1 <= M * topk <= MOE_FUSED_ITEMS.
+bool layout_dispatch_fused(const moe_problem_t& p);
+cudaError_t launch_layout_dispatch(const moe_problem_t& p, const int32_t* topk_idx,
+                                   const int32_t* part_of, const moe_layout_t& lay,
+                                   const void* x, void* recv_x, float* recv_scale,
+                                   cudaStream_t stream);
+
 cudaError_t launch_combine_partial(const moe_problem_t& p, const void* y, const float* w,
                                    const moe_layout_t& lay, void* z, cudaStream_t stream);
 

@@ -209,6 +209,27 @@ int moe_combine(const moe_problem_t *prob, const void *y,
                 moe_stream_t stream);
 
 /*
+ * Layout and dispatch in one call: the same results, bit for bit, as
+ * moe_layout followed by moe_dispatch with the same arguments, and the same
+ * argument rules and return codes as those two calls (workspace included).
+ * Small batches -- 1 <= M*topk <= the library's fused limit (4096 routed
+ * pairs by default), where both steps are bound by latency (Triton-
+ * distributed issue #117, "Results (Latency in us)", M = 2..512) -- run as
+ * ONE kernel in which every block rebuilds the small layout in shared
+ * memory and dispatches its own token, with no inter-block wait; larger
+ * batches run the two calls' kernels.  The workspace is left untouched by
+ * the one-kernel schedule.
+ */
+int moe_layout_dispatch(const moe_problem_t *prob, const int32_t *topk_idx,
+                        const int32_t *part_of, const moe_layout_t *lay,
+                        void *workspace, size_t workspace_bytes, const void *x,
+                        void *recv_x, float *recv_scale, moe_stream_t stream);
+
+/* 1 if moe_layout_dispatch takes the one-kernel schedule for `prob`, else 0
+ * (also 0 for an invalid problem). */
+int moe_layout_dispatch_fused(const moe_problem_t *prob);
+
+/*
  * Two-level combine of a deduplicated dispatch (prob->dedup = 1, else
  * MOE_ERR_ARG): the return path of per-partition dedup, where each
  * partition first reduces the outputs of a token's experts it holds and the

@@ -137,6 +137,33 @@ def test_dispatch_combine_reject_bad_arguments(L):
     assert L.moe_combine_reduce(pd, FAKE, ctypes.byref(lay), FAKE + 8, None) == 1
 
 
+def test_fused_schedule_query(L):
+    """moe_layout_dispatch takes one kernel for small batches only."""
+    f = lambda **kw: L.moe_layout_dispatch_fused(ctypes.byref(P(**kw)))
+    assert f(M=128) == 1 and f(M=1) == 1 and f(M=512) == 1
+    assert f(M=513) == 0 and f(M=4096) == 0 and f(M=0) == 0
+    assert f(M=2048, topk=2) == 1 and f(M=2049, topk=2) == 0
+    assert f(N=12) == 0 and L.moe_layout_dispatch_fused(None) == 0
+
+
+@no_gpu
+def test_layout_dispatch_rejects_bad_arguments(L):
+    lay = fake_layout()
+    ws = L.moe_layout_workspace_size(ctypes.byref(P()))
+    call = lambda prob, idx=FAKE, po=FAKE, lay_=lay, w=FAKE, wb=ws, x=FAKE, r=FAKE, sc=None: \
+        L.moe_layout_dispatch(ctypes.byref(prob), idx, po, ctypes.byref(lay_) if lay_ else None,
+                              w, wb, x, r, sc, None)
+    assert call(P(N=12)) == 1
+    assert call(P(), idx=FAKE + 2) == 1
+    assert call(P(), po=None) == 1
+    assert call(P(), x=FAKE + 8) == 1
+    assert call(P(), r=None) == 1
+    assert call(P(fp8=1)) == 1                       # fp8 needs recv_scale
+    assert call(P(dedup=1), lay_=fake_layout(exp_to_disp=None)) == 1
+    assert call(P(), wb=ws - 1) == 2
+    assert call(P(), w=FAKE + 8) == 2
+
+
 def test_python_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     """No silent fallback: a missing library that cannot be built raises."""
     monkeypatch.setattr(_lib, "_lib", None)
