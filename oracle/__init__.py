@@ -65,6 +65,8 @@ def lib():
                                      ctypes.c_void_p, ctypes.c_void_p]
         L.oracle_combine_partial.restype = ctypes.c_int
         L.oracle_combine_partial.argtypes = [ctypes.c_int32] * 4 + [ctypes.c_int64] + [ctypes.c_void_p] * 8
+        L.oracle_expert_tiles.restype = ctypes.c_int64
+        L.oracle_expert_tiles.argtypes = [ctypes.c_int32, ctypes.c_int32] + [ctypes.c_void_p] * 6
         L.oracle_combine_reduce.restype = ctypes.c_int
         L.oracle_combine_reduce.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int64] + [ctypes.c_void_p] * 4
         _lib = L
@@ -206,6 +208,23 @@ def combine_reduce(z_bits, disp_row, tokens=None):
     if rc != 0:
         raise MemoryError("oracle_combine_reduce: host allocation failed")
     return out
+
+
+def expert_tiles(expert_count, expert_offset, block_m: int) -> dict:
+    """Grouped-GEMM tile metadata of a layout: tile_first [G+1] (per expert,
+    in row order; [G] = number of tiles) and, per tile, tile_expert,
+    tile_row (first row) and tile_rows."""
+    cnt = _c(expert_count, np.int32)
+    off = _c(expert_offset, np.int32)
+    G = cnt.shape[0]
+    if block_m < 1:
+        raise ValueError("block_m must be >= 1")
+    cap = int(sum((int(c) + block_m - 1) // block_m for c in cnt))
+    first = np.zeros(G + 1, np.int32)
+    te, tr, tn = (np.zeros(max(cap, 1), np.int32) for _ in range(3))
+    n = lib().oracle_expert_tiles(G, block_m, _p(cnt), _p(off), _p(first), _p(te), _p(tr), _p(tn))
+    assert n == cap
+    return dict(tile_first=first, tile_expert=te[:n], tile_row=tr[:n], tile_rows=tn[:n], n_tiles=n)
 
 
 def bf16_round(values) -> np.ndarray:

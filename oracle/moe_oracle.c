@@ -30,6 +30,8 @@
  *                element, accumulation in source order.  out[t, c] =
  *                bf16_rne(fma chain over k = 0..topk-1 of
  *                w[t,k] * y[exp_row[t,k], c]) in fp32 starting from +0.
+ *   tiles     -- DeepSpeed PR #8180, "Key points": the per-tile -> group map
+ *                of a grouped GEMM over the expert rows, from the offsets.
  *
  * Invalid input (expert id outside [0, G), placement entry outside
  * [0, E_part)) is never an error of the call: the offending pairs are left out
@@ -433,4 +435,44 @@ int oracle_combine_reduce(int32_t N, int32_t E_part, int64_t n_tok,
     }
     free(acc);
     return 0;
+}
+
+/*
+ * Grouped-GEMM tile metadata (DeepSpeed PR #8180, "Key points": a grouped
+ * GEMM over expert-contiguous rows maps each of its row tiles to a group,
+ * computed from the offsets).  Tiles hold block_m rows and never straddle
+ * two experts: expert e owns n_e = ceil(expert_count[e] / block_m) tiles.
+ * Tiles are numbered in row order, so expert e's first tile is
+ *     tile_first[e] = sum of n_f over the experts f whose rows start before
+ *                     e's (expert_offset[f] < expert_offset[e]),
+ * and tile_first[G] is the number of tiles.  Tile tile_first[e] + j covers
+ * rows [expert_offset[e] + j * block_m, ... + tile_rows) with
+ * tile_rows = min(block_m, expert_count[e] - j * block_m).
+ * Returns the number of tiles; the tile arrays must hold that many.
+ */
+int64_t oracle_expert_tiles(int32_t G, int32_t block_m, const int32_t *expert_count,
+                            const int32_t *expert_offset, int32_t *tile_first,
+                            int32_t *tile_expert, int32_t *tile_row, int32_t *tile_rows)
+{
+    int64_t total = 0;
+    for (int32_t e = 0; e < G; ++e) {
+        int64_t first = 0;
+        for (int32_t f = 0; f < G; ++f)
+            if (expert_offset[f] < expert_offset[e])
+                first += ((int64_t)expert_count[f] + block_m - 1) / block_m;
+        tile_first[e] = (int32_t)first;
+        total += ((int64_t)expert_count[e] + block_m - 1) / block_m;
+    }
+    tile_first[G] = (int32_t)total;
+    for (int32_t e = 0; e < G; ++e) {
+        int64_t n = ((int64_t)expert_count[e] + block_m - 1) / block_m;
+        for (int64_t j = 0; j < n; ++j) {
+            int64_t i = tile_first[e] + j;
+            int64_t rest = expert_count[e] - j * block_m;
+            tile_expert[i] = e;
+            tile_row[i] = (int32_t)(expert_offset[e] + j * block_m);
+            tile_rows[i] = (int32_t)(rest < block_m ? rest : block_m);
+        }
+    }
+    return total;
 }

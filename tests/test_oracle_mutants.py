@@ -19,6 +19,7 @@ from oracle import build as obuild
 import test_oracle_combine as C
 import test_oracle_fp8 as F
 import test_oracle_layout as L
+import test_oracle_tiles as T
 
 SRC = open(obuild.SRC).read()
 
@@ -54,6 +55,14 @@ MUTANTS = [
     ("reduce: drops first partition", "int oracle_combine_reduce", "for (int32_t p = 0; p < E_part; ++p)",
      "for (int32_t p = 1; p < E_part; ++p)"),
     ("reduce: wrong row", "int oracle_combine_reduce", "z + (int64_t)r * N", "z + (int64_t)t * N"),
+    ("tiles: ties before", "int64_t oracle_expert_tiles", "if (expert_offset[f] < expert_offset[e])",
+     "if (expert_offset[f] <= expert_offset[e] && f != e)"),
+    ("tiles: floor count", "int64_t n = ((int64_t)expert_count[e] + block_m - 1) / block_m;",
+     "int64_t n = ((int64_t)expert_count[e] + block_m - 1) / block_m;",
+     "int64_t n = (int64_t)expert_count[e] / block_m;"),
+    ("tiles: full last tile", "int64_t oracle_expert_tiles", "(rest < block_m ? rest : block_m)", "(block_m)"),
+    ("tiles: row start", "int64_t oracle_expert_tiles", "(expert_offset[e] + j * block_m)",
+     "(expert_offset[e] + j * block_m + (j > 0))"),
 ]
 
 
@@ -82,6 +91,9 @@ def _pins():
         lambda: C.test_two_level_one_hot_identity(4),
         lambda: C.test_two_level_colocated_uniform_identity(4),
         lambda: C.test_two_level_within_fp64_bounds(5, 3),
+        lambda: T.test_tiles_match_the_row_walk(1, 8, 2, 1, False, "random", 3),
+        lambda: T.test_tiles_match_the_row_walk(200, 40, 8, 5, True, "random", 16),
+        T.test_block_of_one_row_labels_every_row,
     ]
 
 
