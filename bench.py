@@ -308,37 +308,38 @@ def run_ours(args, w):
         raise SystemExit("--combine two-level needs a dedup workload")
     separate = args.schedule == "separate"
     fused = not separate and moe.moe_layout_dispatch_fused(prob)
+    bm = args.tiles or None
     # eager warm-up through the public API, then one graph per step with
     # external events between the kernels
     with torch.cuda.stream(stream):
         for _ in range(3):
-            buf.step(idx, po, x, y, gates, two_level=two_level, separate=separate)
+            buf.step(idx, po, x, y, gates, two_level=two_level, separate=separate, block_m=bm)
     stream.synchronize()
+    # the step's parts in launch order (the tile metadata, when asked for,
+    # comes where a grouped GEMM would consume it: after the dispatch)
+    parts = ([("layout+dispatch", lambda: buf.layout_dispatch_(idx, po, x))] if fused else
+             [("layout", lambda: buf.layout_(idx, po)), ("dispatch", lambda: buf.dispatch_(x))])
+    if bm:
+        parts.append(("tiles", lambda: buf.expert_tiles_(po, bm)))
+    # the two-level combine is two kernels: one interval covers the pair
+    parts.append(("combine", (lambda: buf.combine_two_level_(y, gates)) if two_level else
+                  (lambda: buf.combine_(y, gates))))
+
     # Two graphs of the same step.  The timed one has events only at its two
     # ends, so consecutive kernels keep their programmatic (early-launch)
-    # edges as in production; the second has events between the kernels for
+    # edges as in production; the second has events between the parts for
     # the per-kernel breakdown (an event node between two kernels replaces
     # that edge with a full dependency, so its parts add up to a little more
     # than the step).
     def capture(inner):
-        ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
-        mark = (lambda i: ev[i].record()) if inner else (lambda i: None)
+        ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(parts) + 1)]
         graph = torch.cuda.CUDAGraph(keep_graph=True)
         with torch.cuda.graph(graph, stream=stream):
             ev[0].record()
-            if fused:  # one kernel: layout and dispatch share one interval
-                buf.layout_dispatch_(idx, po, x)
-                mark(1)
-            else:
-                buf.layout_(idx, po)
-                mark(1)
-                buf.dispatch_(x)
-            mark(2)
-            if two_level:
-                buf.combine_two_level_(y, gates)  # two kernels: events only around the pair
-            else:
-                buf.combine_(y, gates)
-            ev[3].record()
+            for i, (_, fn) in enumerate(parts):
+                fn()
+                if inner or i == len(parts) - 1:
+                    ev[i + 1].record()
         n = graph_kernel_nodes(graph)
         graph.instantiate()
         return graph, ev, n
@@ -350,13 +351,15 @@ def run_ours(args, w):
     status = int(buf.layout.status.item())
     if status:
         raise SystemExit(f"layout status {status}")
-    abytes = algorithmic_bytes(wr, R_exp, R_disp, two_level)
-    if two_level:  # one timed interval covers both combine kernels
-        abytes = {"layout": abytes["layout"], "dispatch": abytes["dispatch"],
-                  "combine": abytes["combine_partial"] + abytes["combine_reduce"]}
+    ab = algorithmic_bytes(wr, R_exp, R_disp, two_level)
+    if two_level:
+        ab["combine"] = ab.pop("combine_partial") + ab.pop("combine_reduce")
     if fused:
-        abytes = {"layout+dispatch": abytes["layout"] + abytes["dispatch"],
-                  "combine": abytes["combine"]}
+        ab["layout+dispatch"] = ab.pop("layout") + ab.pop("dispatch")
+    if bm:
+        n_tiles = int(buf.tiles.tile_first[w.G].item())
+        ab["tiles"] = 4 * (3 * w.G + w.G + 1) + 12 * n_tiles
+    abytes = {name: ab[name] for name, _ in parts}
     step_bytes = sum(abytes.values())
     move = "layout+dispatch" if fused else "dispatch"
 
@@ -365,15 +368,14 @@ def run_ours(args, w):
             flush()
             graph.replay()
         stream.synchronize()
-        return ev[0].elapsed_time(ev[3])
+        return ev[0].elapsed_time(ev[-1])
 
     def parts_step():
         with torch.cuda.stream(stream):
             flush()
             pgraph.replay()
         stream.synchronize()
-        return (pev[0].elapsed_time(pev[3]), pev[0].elapsed_time(pev[1]),
-                pev[1].elapsed_time(pev[2]), pev[2].elapsed_time(pev[3]))
+        return [pev[i].elapsed_time(pev[i + 1]) for i in range(len(parts))]
 
     for _ in range(max(args.warmup, 3)):
         timed_step()
@@ -391,16 +393,12 @@ def run_ours(args, w):
     # per-kernel breakdown (untimed for the headline; same flush, same inputs)
     for _ in range(3):
         parts_step()
-    per = np.array([parts_step() for _ in range(args.steps)])   # [K, 4] ms
-    if fused:
-        kern_ms = {"layout+dispatch": float(per[:, 1].mean()), "combine": float(per[:, 3].mean())}
-    else:
-        kern_ms = {"layout": float(per[:, 1].mean()), "dispatch": float(per[:, 2].mean()),
-                   "combine": float(per[:, 3].mean())}
+    per = np.array([parts_step() for _ in range(args.steps)])   # [K, parts] ms
+    kern_ms = {name: float(per[:, i].mean()) for i, (name, _) in enumerate(parts)}
 
     # end to end through the public API with host buffers
     e2e = run_e2e(args, wr, buf, idx_h, po_h, g_h, x, y, stream, dev, flush, step_bytes,
-                  two_level, separate)
+                  two_level, separate, bm)
 
     # aggregate over ranks: bytes and tokens summed, time = max
     (max_ms, max_e2e_ms), (all_bytes, all_tokens, all_e2e_bytes) = reduce_over_ranks(
@@ -413,6 +411,7 @@ def run_ours(args, w):
         ach = abytes[dom] / (kern_ms[dom] * 1e-3) / 1e9
         kern_names = {"dispatch": "dispatch_fp8_kernel" if w.fp8 else "dispatch_bf16_kernel",
                       "layout+dispatch": "layout_dispatch_kernel",
+                      "tiles": "expert_tiles_kernel",
                       "combine": "combine_partial_kernel+combine_reduce_kernel" if two_level
                       else "combine_kernel"}
         line = {
@@ -427,6 +426,7 @@ def run_ours(args, w):
                 "combine": "two-level (per partition, then per token)" if two_level else "one-level",
                 "schedule": "one kernel for layout + dispatch" if fused else
                             "separate layout and dispatch kernels",
+                "tiles_block_m": bm,
                 "l2": "flushed between timed steps (256 MiB write + 256 MiB read, untimed)",
                 "timing": "one CUDA graph replay per step; CUDA events recorded inside the graph "
                           "on the launch stream at its start and end"}),
@@ -462,7 +462,7 @@ def run_ours(args, w):
 
 
 def run_e2e(args, w, buf, idx_h, po_h, g_h, x, y, stream, dev, flush, step_bytes,
-            two_level=False, separate=False):
+            two_level=False, separate=False, block_m=None):
     """Public-API calls on host inputs: pinned host -> device copies of every
     input, layout / dispatch / combine, device -> host copy of the output."""
     import torch
@@ -488,7 +488,8 @@ def run_e2e(args, w, buf, idx_h, po_h, g_h, x, y, stream, dev, flush, step_bytes
             s.record()
             for dst, src in ((d_idx, hidx), (d_po, hpo), (d_g, hg), (d_x, hx), (d_y, hy)):
                 dst.copy_(src, non_blocking=True)
-            out = buf.step(d_idx, d_po, d_x, d_y, d_g, two_level=two_level, separate=separate)
+            out = buf.step(d_idx, d_po, d_x, d_y, d_g, two_level=two_level, separate=separate,
+                           block_m=block_m)
             hout.copy_(out, non_blocking=True)
             e.record()
         e.synchronize()
@@ -604,6 +605,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--schedule", choices=("auto", "separate"), default="auto",
                     help="separate: moe_layout + moe_dispatch even where one kernel does both")
+    ap.add_argument("--tiles", type=int, default=0, metavar="BM",
+                    help="also build the grouped-GEMM tile metadata (tiles of BM rows) each step")
     ap.add_argument("--combine", choices=("one-level", "two-level"), default="one-level",
                     help="two-level: per-partition reduce then per-token sum (dedup workloads)")
     ap.add_argument("--latency-sweep", action="store_true",

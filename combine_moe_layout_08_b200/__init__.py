@@ -28,7 +28,8 @@ from ._lib import (MOE_MAX_E_PART, MOE_MAX_G, MOE_MAX_TOPK, MOE_STATIC_SCRATCH_B
 
 __all__ = ["MoEProblem", "MoELayout", "MoEBuffers", "MoEError", "alloc_layout",
            "layout_workspace_size", "moe_layout", "moe_layout_static", "moe_dispatch",
-           "moe_layout_dispatch", "moe_layout_dispatch_fused", "moe_combine", "moe_combine_partial", "moe_combine_reduce",
+           "moe_layout_dispatch", "moe_layout_dispatch_fused", "moe_expert_tiles",
+           "expert_tiles_capacity", "alloc_expert_tiles", "ExpertTiles", "moe_combine", "moe_combine_partial", "moe_combine_reduce",
            "moe_status_string", "moe_abi_version", "MOE_STATUS_BAD_EXPERT",
            "MOE_STATUS_BAD_PART", "MOE_STATUS_BAD_ROW", "MOE_MAX_G", "MOE_MAX_E_PART",
            "MOE_MAX_TOPK"]
@@ -219,6 +220,51 @@ def moe_layout_dispatch_fused(prob: MoEProblem) -> bool:
     return bool(_lib.load().moe_layout_dispatch_fused(ctypes.byref(s)))
 
 
+def expert_tiles_capacity(prob: MoEProblem, block_m: int) -> int:
+    """Entries each tile array of moe_expert_tiles needs (0: invalid)."""
+    s = prob.struct()
+    return int(_lib.load().moe_expert_tiles_capacity(ctypes.byref(s), block_m))
+
+
+@dataclasses.dataclass
+class ExpertTiles:
+    """Grouped-GEMM tile metadata on the device (see moe_expert_tiles)."""
+    block_m: int
+    tile_first: torch.Tensor   # [G+1] int32
+    tile_expert: torch.Tensor  # [cap] int32
+    tile_row: torch.Tensor     # [cap] int32
+    tile_rows: torch.Tensor    # [cap] int32
+
+
+def alloc_expert_tiles(prob: MoEProblem, block_m: int, device) -> ExpertTiles:
+    cap = expert_tiles_capacity(prob, block_m)
+    if cap == 0:
+        raise ValueError(f"invalid problem or block_m={block_m}")
+    i32 = dict(dtype=torch.int32, device=device)
+    return ExpertTiles(block_m, torch.empty(prob.G + 1, **i32), torch.empty(cap, **i32),
+                       torch.empty(cap, **i32), torch.empty(cap, **i32))
+
+
+def moe_expert_tiles(prob: MoEProblem, part_of: torch.Tensor, lay: MoELayout,
+                     tiles: ExpertTiles, stream=None) -> None:
+    """Per-tile expert map of a grouped GEMM over the layout's expert rows,
+    tiles of ``tiles.block_m`` rows in row order (after moe_layout)."""
+    dev = part_of.device
+    cap = expert_tiles_capacity(prob, tiles.block_m)
+    _check(part_of, "part_of", torch.int32, prob.G, dev)
+    _check(tiles.tile_first, "tile_first", torch.int32, prob.G + 1, dev)
+    for name in ("tile_expert", "tile_row", "tile_rows"):
+        _check(getattr(tiles, name), name, torch.int32, cap, dev)
+    _check_layout(prob, lay, dev)
+    s, l = prob.struct(), lay.struct()
+    rc = _lib.load().moe_expert_tiles(
+        ctypes.byref(s), part_of.data_ptr(), ctypes.byref(l), tiles.block_m,
+        tiles.tile_first.data_ptr(), tiles.tile_expert.data_ptr(), tiles.tile_row.data_ptr(),
+        tiles.tile_rows.data_ptr(), _stream(part_of, stream))
+    if rc:
+        raise MoEError("moe_expert_tiles", rc)
+
+
 def moe_combine(prob: MoEProblem, y: torch.Tensor, topk_weights: torch.Tensor, lay: MoELayout,
                 out: torch.Tensor, stream=None) -> None:
     """out [M, N] bf16 = gate-weighted sum of the expert rows ``y`` [M*topk, N] bf16."""
@@ -310,15 +356,27 @@ class MoEBuffers:
         moe_combine_partial(self.prob, y, topk_weights, self.layout, self.z, stream)
         moe_combine_reduce(self.prob, self.z, self.layout, self.out, stream)
 
+    def expert_tiles_(self, part_of, block_m, stream=None):
+        """Grouped-GEMM tile metadata of the current layout into ``self.tiles``
+        (allocated on first use, or when block_m changes)."""
+        t = getattr(self, "tiles", None)
+        if t is None or t.block_m != block_m:
+            self.tiles = t = alloc_expert_tiles(self.prob, block_m, self.device)
+        moe_expert_tiles(self.prob, part_of, self.layout, t, stream)
+
     def step(self, topk_idx, part_of, x, y, topk_weights, stream=None, two_level=False,
-             separate=False):
+             separate=False, block_m=None):
         """layout -> dispatch -> combine; ``separate`` calls moe_layout and
-        moe_dispatch instead of moe_layout_dispatch (same results)."""
+        moe_dispatch instead of moe_layout_dispatch (same results);
+        ``block_m`` also builds the grouped-GEMM tile metadata after the
+        dispatch."""
         if separate:
             self.layout_(topk_idx, part_of, stream)
             self.dispatch_(x, stream)
         else:
             self.layout_dispatch_(topk_idx, part_of, x, stream)
+        if block_m:
+            self.expert_tiles_(part_of, block_m, stream)
         if two_level:
             self.combine_two_level_(y, topk_weights, stream)
         else:

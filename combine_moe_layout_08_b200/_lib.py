@@ -59,6 +59,11 @@ SIGNATURES = {
                                            ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
                                            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "moe_layout_dispatch_fused": (ctypes.c_int, [ctypes.POINTER(ProblemStruct)]),
+    "moe_expert_tiles_capacity": (ctypes.c_size_t, [ctypes.POINTER(ProblemStruct), ctypes.c_int32]),
+    "moe_expert_tiles": (ctypes.c_int, [ctypes.POINTER(ProblemStruct), ctypes.c_void_p,
+                                        ctypes.POINTER(LayoutStruct), ctypes.c_int32,
+                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                        ctypes.c_void_p, ctypes.c_void_p]),
     "moe_combine": (ctypes.c_int, [ctypes.POINTER(ProblemStruct), ctypes.c_void_p, ctypes.c_void_p,
                                    ctypes.POINTER(LayoutStruct), ctypes.c_void_p, ctypes.c_void_p]),
     "moe_combine_partial": (ctypes.c_int, [ctypes.POINTER(ProblemStruct), ctypes.c_void_p,

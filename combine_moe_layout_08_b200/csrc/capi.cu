@@ -105,6 +105,23 @@ int moe_layout_dispatch(const moe_problem_t* prob, const int32_t* topk_idx,
   return cuda_rc(moe::launch_dispatch(*prob, x, *lay, recv_x, recv_scale, s));
 }
 
+size_t moe_expert_tiles_capacity(const moe_problem_t* prob, int32_t block_m) {
+  if (!valid_problem(prob) || block_m < 1) return 0;
+  return (size_t)moe::expert_tiles_capacity(*prob, block_m);
+}
+
+int moe_expert_tiles(const moe_problem_t* prob, const int32_t* part_of, const moe_layout_t* lay,
+                     int32_t block_m, int32_t* tile_first, int32_t* tile_expert,
+                     int32_t* tile_row, int32_t* tile_rows, moe_stream_t stream) {
+  if (!valid_problem(prob) || !valid_layout(prob, lay) || block_m < 1) return MOE_ERR_ARG;
+  if (!arr(part_of) || !arr(tile_first) || !arr(tile_expert) || !arr(tile_row) || !arr(tile_rows))
+    return MOE_ERR_ARG;
+  if (moe::expert_tiles_capacity(*prob, block_m) >= ((int64_t)1 << 31)) return MOE_ERR_ARG;
+  return cuda_rc(moe::launch_expert_tiles(*prob, part_of, *lay, block_m, tile_first, tile_expert,
+                                          tile_row, tile_rows,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int moe_combine(const moe_problem_t* prob, const void* y, const float* topk_weights,
                 const moe_layout_t* lay, void* out, moe_stream_t stream) {
   if (!valid_problem(prob) || !valid_layout(prob, lay)) return MOE_ERR_ARG;

@@ -66,6 +66,13 @@ cudaError_t launch_layout_dispatch(const moe_problem_t& p, const int32_t* topk_i
                                    const void* x, void* recv_x, float* recv_scale,
                                    cudaStream_t stream);
 
+// Grouped-GEMM tile metadata of a layout (entries per tile array: capacity).
+int64_t expert_tiles_capacity(const moe_problem_t& p, int block_m);
+cudaError_t launch_expert_tiles(const moe_problem_t& p, const int32_t* part_of,
+                                const moe_layout_t& lay, int block_m, int32_t* tile_first,
+                                int32_t* tile_expert, int32_t* tile_row, int32_t* tile_rows,
+                                cudaStream_t stream);
+
 cudaError_t launch_combine_partial(const moe_problem_t& p, const void* y, const float* w,
                                    const moe_layout_t& lay, void* z, cudaStream_t stream);
 

@@ -230,6 +230,32 @@ int moe_layout_dispatch(const moe_problem_t *prob, const int32_t *topk_idx,
 int moe_layout_dispatch_fused(const moe_problem_t *prob);
 
 /*
+ * Grouped-GEMM tile metadata of a layout, computed on the device so that a
+ * grouped GEMM over the expert rows needs no device -> host copy of the
+ * offsets (DeepSpeed PR #8180, "Key points": per-tile -> group mapping
+ * computed on device from offs).  Tiles hold block_m rows and never
+ * straddle two experts: expert e owns ceil(expert_count[e] / block_m)
+ * tiles, numbered in row order.  Call after moe_layout (same stream) with
+ * the same part_of.
+ *   tile_first  [G+1] int32: first tile of expert e (also defined for
+ *               experts without rows); tile_first[G] = number of tiles
+ *   tile_expert [cap] int32: expert of tile i
+ *   tile_row    [cap] int32: first expert row of tile i
+ *   tile_rows   [cap] int32: rows of tile i, 1..block_m
+ * cap = moe_expert_tiles_capacity(prob, block_m) = ceil(M*topk/block_m) + G
+ * entries, the most a layout of this problem needs; entries past
+ * tile_first[G] are untouched.  Counts that cannot come from a layout of
+ * this problem (more tiles than cap) write cap tiles and raise
+ * MOE_STATUS_BAD_ROW.  MOE_ERR_ARG for block_m < 1, a capacity of 2^31 or
+ * more, or null / misaligned arrays.
+ */
+size_t moe_expert_tiles_capacity(const moe_problem_t *prob, int32_t block_m);
+int moe_expert_tiles(const moe_problem_t *prob, const int32_t *part_of,
+                     const moe_layout_t *lay, int32_t block_m,
+                     int32_t *tile_first, int32_t *tile_expert,
+                     int32_t *tile_row, int32_t *tile_rows, moe_stream_t stream);
+
+/*
  * Two-level combine of a deduplicated dispatch (prob->dedup = 1, else
  * MOE_ERR_ARG): the return path of per-partition dedup, where each
  * partition first reduces the outputs of a token's experts it holds and the

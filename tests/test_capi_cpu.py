@@ -164,6 +164,26 @@ def test_layout_dispatch_rejects_bad_arguments(L):
     assert call(P(), w=FAKE + 8) == 2
 
 
+def test_expert_tiles_capacity(L):
+    cap = lambda bm, **kw: L.moe_expert_tiles_capacity(ctypes.byref(P(**kw)), bm)
+    assert cap(128) == (128 * 8 + 127) // 128 + 256
+    assert cap(1) == 128 * 8 + 256
+    assert cap(0) == 0 and cap(-3) == 0 and cap(128, N=12) == 0
+    assert cap(7, M=0) == 256
+
+
+@no_gpu
+def test_expert_tiles_rejects_bad_arguments(L):
+    lay = fake_layout()
+    p = ctypes.byref(P())
+    ok = (FAKE, FAKE + 64, FAKE + 128, FAKE + 192)
+    assert L.moe_expert_tiles(p, FAKE, ctypes.byref(lay), 0, *ok, None) == 1
+    assert L.moe_expert_tiles(p, None, ctypes.byref(lay), 64, *ok, None) == 1
+    assert L.moe_expert_tiles(p, FAKE, None, 64, *ok, None) == 1
+    assert L.moe_expert_tiles(p, FAKE, ctypes.byref(lay), 64, FAKE, FAKE + 2, FAKE, FAKE, None) == 1
+    assert L.moe_expert_tiles(p, FAKE, ctypes.byref(lay), 64, FAKE, FAKE, FAKE, None, None) == 1
+
+
 def test_python_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     """No silent fallback: a missing library that cannot be built raises."""
     monkeypatch.setattr(_lib, "_lib", None)
