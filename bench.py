@@ -315,11 +315,17 @@ def run_ours(args, w):
         for _ in range(3):
             buf.step(idx, po, x, y, gates, two_level=two_level, separate=separate, block_m=bm)
     stream.synchronize()
-    # the step's parts in launch order (the tile metadata, when asked for,
-    # comes where a grouped GEMM would consume it: after the dispatch)
-    parts = ([("layout+dispatch", lambda: buf.layout_dispatch_(idx, po, x))] if fused else
-             [("layout", lambda: buf.layout_(idx, po)), ("dispatch", lambda: buf.dispatch_(x))])
-    if bm:
+    # the step's parts in launch order.  The grouped-GEMM tile metadata, when
+    # asked for, comes out of moe_layout_dispatch's own kernels (one part,
+    # whatever the schedule), or with --schedule separate from its own
+    # kernel after the dispatch.
+    if bm and not separate:
+        parts = [("layout+dispatch", lambda: buf.layout_dispatch_(idx, po, x, block_m=bm))]
+    elif fused:
+        parts = [("layout+dispatch", lambda: buf.layout_dispatch_(idx, po, x))]
+    else:
+        parts = [("layout", lambda: buf.layout_(idx, po)), ("dispatch", lambda: buf.dispatch_(x))]
+    if bm and separate:
         parts.append(("tiles", lambda: buf.expert_tiles_(po, bm)))
     # the two-level combine is two kernels: one interval covers the pair
     parts.append(("combine", (lambda: buf.combine_two_level_(y, gates)) if two_level else
@@ -354,14 +360,15 @@ def run_ours(args, w):
     ab = algorithmic_bytes(wr, R_exp, R_disp, two_level)
     if two_level:
         ab["combine"] = ab.pop("combine_partial") + ab.pop("combine_reduce")
-    if fused:
-        ab["layout+dispatch"] = ab.pop("layout") + ab.pop("dispatch")
     if bm:
         n_tiles = int(buf.tiles.tile_first[w.G].item())
         ab["tiles"] = 4 * (3 * w.G + w.G + 1) + 12 * n_tiles
+    if parts[0][0] == "layout+dispatch":
+        ab["layout+dispatch"] = ab.pop("layout") + ab.pop("dispatch") + \
+            (ab.pop("tiles") if bm and not separate else 0)
     abytes = {name: ab[name] for name, _ in parts}
     step_bytes = sum(abytes.values())
-    move = "layout+dispatch" if fused else "dispatch"
+    move = parts[0][0] if parts[0][0] == "layout+dispatch" else "dispatch"
 
     def timed_step():
         with torch.cuda.stream(stream):
@@ -410,7 +417,8 @@ def run_ours(args, w):
         dom = max((move, "combine"), key=lambda k: kern_ms[k])
         ach = abytes[dom] / (kern_ms[dom] * 1e-3) / 1e9
         kern_names = {"dispatch": "dispatch_fp8_kernel" if w.fp8 else "dispatch_bf16_kernel",
-                      "layout+dispatch": "layout_dispatch_kernel",
+                      "layout+dispatch": "layout_dispatch_kernel" if fused else
+                      "layout kernels+" + ("dispatch_fp8_kernel" if w.fp8 else "dispatch_bf16_kernel"),
                       "tiles": "expert_tiles_kernel",
                       "combine": "combine_partial_kernel+combine_reduce_kernel" if two_level
                       else "combine_kernel"}
@@ -424,7 +432,7 @@ def run_ours(args, w):
             "config": config_of(w, extra={
                 "R_exp": R_exp, "R_disp": R_disp,
                 "combine": "two-level (per partition, then per token)" if two_level else "one-level",
-                "schedule": "one kernel for layout + dispatch" if fused else
+                "schedule": "one kernel for layout + dispatch" if fused and not separate else
                             "separate layout and dispatch kernels",
                 "tiles_block_m": bm,
                 "l2": "flushed between timed steps (256 MiB write + 256 MiB read, untimed)",

@@ -192,9 +192,10 @@ def moe_dispatch(prob: MoEProblem, x: torch.Tensor, lay: MoELayout, recv_x: torc
 def moe_layout_dispatch(prob: MoEProblem, topk_idx: torch.Tensor, part_of: torch.Tensor,
                         lay: MoELayout, workspace: torch.Tensor, x: torch.Tensor,
                         recv_x: torch.Tensor, recv_scale: Optional[torch.Tensor] = None,
-                        stream=None) -> None:
+                        tiles: Optional["ExpertTiles"] = None, stream=None) -> None:
     """moe_layout then moe_dispatch in one call (bit-identical results); small
-    batches run as one kernel (see ``moe_layout_dispatch_fused``)."""
+    batches run as one kernel (see ``moe_layout_dispatch_fused``).  ``tiles``
+    also fills the grouped-GEMM tile metadata from the same kernels."""
     dev = x.device
     cap = prob.capacity
     _check(topk_idx, "topk_idx", torch.int32, prob.M * prob.topk, dev)
@@ -205,11 +206,15 @@ def moe_layout_dispatch(prob: MoEProblem, topk_idx: torch.Tensor, part_of: torch
     if prob.fp8:
         _check(recv_scale, "recv_scale", torch.float32, cap * (prob.N // 128), dev)
     _check_layout(prob, lay, dev)
+    if tiles is not None:
+        _check_tiles(prob, tiles, dev)
     s, l = prob.struct(), lay.struct()
+    ts = tiles.struct() if tiles is not None else None
     rc = _lib.load().moe_layout_dispatch(
         ctypes.byref(s), topk_idx.data_ptr(), part_of.data_ptr(), ctypes.byref(l),
         workspace.data_ptr(), workspace.numel(), x.data_ptr(), recv_x.data_ptr(),
-        recv_scale.data_ptr() if recv_scale is not None else None, _stream(x, stream))
+        recv_scale.data_ptr() if recv_scale is not None else None,
+        ctypes.byref(ts) if ts is not None else None, _stream(x, stream))
     if rc:
         raise MoEError("moe_layout_dispatch", rc)
 
@@ -235,6 +240,20 @@ class ExpertTiles:
     tile_row: torch.Tensor     # [cap] int32
     tile_rows: torch.Tensor    # [cap] int32
 
+    def struct(self) -> _lib.TilesStruct:
+        return _lib.TilesStruct(self.block_m, self.tile_first.data_ptr(),
+                                self.tile_expert.data_ptr(), self.tile_row.data_ptr(),
+                                self.tile_rows.data_ptr())
+
+
+def _check_tiles(prob: MoEProblem, tiles: ExpertTiles, device):
+    cap = expert_tiles_capacity(prob, tiles.block_m)
+    if cap == 0:
+        raise ValueError(f"invalid block_m={tiles.block_m}")
+    _check(tiles.tile_first, "tile_first", torch.int32, prob.G + 1, device)
+    for name in ("tile_expert", "tile_row", "tile_rows"):
+        _check(getattr(tiles, name), name, torch.int32, cap, device)
+
 
 def alloc_expert_tiles(prob: MoEProblem, block_m: int, device) -> ExpertTiles:
     cap = expert_tiles_capacity(prob, block_m)
@@ -250,17 +269,12 @@ def moe_expert_tiles(prob: MoEProblem, part_of: torch.Tensor, lay: MoELayout,
     """Per-tile expert map of a grouped GEMM over the layout's expert rows,
     tiles of ``tiles.block_m`` rows in row order (after moe_layout)."""
     dev = part_of.device
-    cap = expert_tiles_capacity(prob, tiles.block_m)
     _check(part_of, "part_of", torch.int32, prob.G, dev)
-    _check(tiles.tile_first, "tile_first", torch.int32, prob.G + 1, dev)
-    for name in ("tile_expert", "tile_row", "tile_rows"):
-        _check(getattr(tiles, name), name, torch.int32, cap, dev)
+    _check_tiles(prob, tiles, dev)
     _check_layout(prob, lay, dev)
-    s, l = prob.struct(), lay.struct()
-    rc = _lib.load().moe_expert_tiles(
-        ctypes.byref(s), part_of.data_ptr(), ctypes.byref(l), tiles.block_m,
-        tiles.tile_first.data_ptr(), tiles.tile_expert.data_ptr(), tiles.tile_row.data_ptr(),
-        tiles.tile_rows.data_ptr(), _stream(part_of, stream))
+    s, l, ts = prob.struct(), lay.struct(), tiles.struct()
+    rc = _lib.load().moe_expert_tiles(ctypes.byref(s), part_of.data_ptr(), ctypes.byref(l),
+                                      ctypes.byref(ts), _stream(part_of, stream))
     if rc:
         raise MoEError("moe_expert_tiles", rc)
 
@@ -340,9 +354,18 @@ class MoEBuffers:
     def dispatch_(self, x, stream=None):
         moe_dispatch(self.prob, x, self.layout, self.recv_x, self.recv_scale, stream)
 
-    def layout_dispatch_(self, topk_idx, part_of, x, stream=None):
+    def _tiles_for(self, block_m):
+        t = getattr(self, "tiles", None)
+        if t is None or t.block_m != block_m:
+            self.tiles = t = alloc_expert_tiles(self.prob, block_m, self.device)
+        return t
+
+    def layout_dispatch_(self, topk_idx, part_of, x, stream=None, block_m=None):
+        """moe_layout_dispatch; ``block_m`` also fills ``self.tiles`` from the
+        same kernels."""
         moe_layout_dispatch(self.prob, topk_idx, part_of, self.layout, self.workspace, x,
-                            self.recv_x, self.recv_scale, stream)
+                            self.recv_x, self.recv_scale,
+                            self._tiles_for(block_m) if block_m else None, stream)
 
     def combine_(self, y, topk_weights, stream=None):
         moe_combine(self.prob, y, topk_weights, self.layout, self.out, stream)
@@ -358,25 +381,22 @@ class MoEBuffers:
 
     def expert_tiles_(self, part_of, block_m, stream=None):
         """Grouped-GEMM tile metadata of the current layout into ``self.tiles``
-        (allocated on first use, or when block_m changes)."""
-        t = getattr(self, "tiles", None)
-        if t is None or t.block_m != block_m:
-            self.tiles = t = alloc_expert_tiles(self.prob, block_m, self.device)
-        moe_expert_tiles(self.prob, part_of, self.layout, t, stream)
+        by its own kernel (allocated on first use, or when block_m changes)."""
+        moe_expert_tiles(self.prob, part_of, self.layout, self._tiles_for(block_m), stream)
 
     def step(self, topk_idx, part_of, x, y, topk_weights, stream=None, two_level=False,
              separate=False, block_m=None):
         """layout -> dispatch -> combine; ``separate`` calls moe_layout and
         moe_dispatch instead of moe_layout_dispatch (same results);
-        ``block_m`` also builds the grouped-GEMM tile metadata after the
-        dispatch."""
+        ``block_m`` also builds the grouped-GEMM tile metadata (inside
+        moe_layout_dispatch, or by moe_expert_tiles after separate calls)."""
         if separate:
             self.layout_(topk_idx, part_of, stream)
             self.dispatch_(x, stream)
+            if block_m:
+                self.expert_tiles_(part_of, block_m, stream)
         else:
-            self.layout_dispatch_(topk_idx, part_of, x, stream)
-        if block_m:
-            self.expert_tiles_(part_of, block_m, stream)
+            self.layout_dispatch_(topk_idx, part_of, x, stream, block_m)
         if two_level:
             self.combine_two_level_(y, topk_weights, stream)
         else:

@@ -41,6 +41,11 @@ class LayoutStruct(ctypes.Structure):
 
 
 # exported symbol -> (restype, argtypes)
+class TilesStruct(ctypes.Structure):
+    _fields_ = [("block_m", ctypes.c_int32)] + [
+        (n, ctypes.c_void_p) for n in ("tile_first", "tile_expert", "tile_row", "tile_rows")]
+
+
 SIGNATURES = {
     "moe_abi_version": (ctypes.c_int, []),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -57,13 +62,13 @@ SIGNATURES = {
     "moe_layout_dispatch": (ctypes.c_int, [ctypes.POINTER(ProblemStruct), ctypes.c_void_p,
                                            ctypes.c_void_p, ctypes.POINTER(LayoutStruct),
                                            ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
-                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+                                           ctypes.c_void_p, ctypes.c_void_p,
+                                           ctypes.POINTER(TilesStruct), ctypes.c_void_p]),
     "moe_layout_dispatch_fused": (ctypes.c_int, [ctypes.POINTER(ProblemStruct)]),
     "moe_expert_tiles_capacity": (ctypes.c_size_t, [ctypes.POINTER(ProblemStruct), ctypes.c_int32]),
     "moe_expert_tiles": (ctypes.c_int, [ctypes.POINTER(ProblemStruct), ctypes.c_void_p,
-                                        ctypes.POINTER(LayoutStruct), ctypes.c_int32,
-                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
-                                        ctypes.c_void_p, ctypes.c_void_p]),
+                                        ctypes.POINTER(LayoutStruct), ctypes.POINTER(TilesStruct),
+                                        ctypes.c_void_p]),
     "moe_combine": (ctypes.c_int, [ctypes.POINTER(ProblemStruct), ctypes.c_void_p, ctypes.c_void_p,
                                    ctypes.POINTER(LayoutStruct), ctypes.c_void_p, ctypes.c_void_p]),
     "moe_combine_partial": (ctypes.c_int, [ctypes.POINTER(ProblemStruct), ctypes.c_void_p,

@@ -3,6 +3,7 @@
 // launches.  See include/moe_layout.h for the contract of each call.
 #include <cstdint>
 
+#include "layout_device.cuh"
 #include "moe_internal.h"
 #include "moe_layout.h"
 
@@ -37,6 +38,27 @@ bool valid_layout(const moe_problem_t* p, const moe_layout_t* l) {
 
 int cuda_rc(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
+// tile metadata request: block_m >= 1, arrays present and aligned, capacity
+// below 2^31 entries
+bool valid_tiles(const moe_problem_t* p, const moe_tiles_t* t) {
+  if (!t || t->block_m < 1) return false;
+  if (!arr(t->tile_first) || !arr(t->tile_expert) || !arr(t->tile_row) || !arr(t->tile_rows))
+    return false;
+  return moe::expert_tiles_capacity(*p, t->block_m) < ((int64_t)1 << 31);
+}
+
+moe::TileOut tile_out(const moe_tiles_t* t) {
+  moe::TileOut o{};
+  if (t) {
+    o.block_m = t->block_m;
+    o.tile_first = t->tile_first;
+    o.tile_expert = t->tile_expert;
+    o.tile_row = t->tile_row;
+    o.tile_rows = t->tile_rows;
+  }
+  return o;
+}
+
 }  // namespace
 
 extern "C" {
@@ -66,7 +88,7 @@ int moe_layout(const moe_problem_t* prob, const int32_t* topk_idx, const int32_t
   const size_t need = moe::layout_workspace_bytes(*prob);
   if (!workspace || !aligned(workspace, 16) || workspace_bytes < need) return MOE_ERR_WORKSPACE;
   return cuda_rc(moe::launch_layout(*prob, topk_idx, part_of, *lay, workspace,
-                                    reinterpret_cast<cudaStream_t>(stream)));
+                                    reinterpret_cast<cudaStream_t>(stream), moe::TileOut{}));
 }
 
 int moe_dispatch(const moe_problem_t* prob, const void* x, const moe_layout_t* lay,
@@ -87,8 +109,9 @@ int moe_layout_dispatch_fused(const moe_problem_t* prob) {
 int moe_layout_dispatch(const moe_problem_t* prob, const int32_t* topk_idx,
                         const int32_t* part_of, const moe_layout_t* lay, void* workspace,
                         size_t workspace_bytes, const void* x, void* recv_x, float* recv_scale,
-                        moe_stream_t stream) {
+                        const moe_tiles_t* tiles, moe_stream_t stream) {
   if (!valid_problem(prob) || !valid_layout(prob, lay)) return MOE_ERR_ARG;
+  if (tiles && !valid_tiles(prob, tiles)) return MOE_ERR_ARG;
   if (!arr(part_of) || (prob->M > 0 && !arr(topk_idx))) return MOE_ERR_ARG;
   if (prob->M > 0) {
     if (!x || !aligned(x, 16) || !recv_x || !aligned(recv_x, 16)) return MOE_ERR_ARG;
@@ -97,10 +120,11 @@ int moe_layout_dispatch(const moe_problem_t* prob, const int32_t* topk_idx,
   const size_t need = moe::layout_workspace_bytes(*prob);
   if (!workspace || !aligned(workspace, 16) || workspace_bytes < need) return MOE_ERR_WORKSPACE;
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const moe::TileOut t = tile_out(tiles);
   if (moe::layout_dispatch_fused(*prob))
     return cuda_rc(moe::launch_layout_dispatch(*prob, topk_idx, part_of, *lay, x, recv_x,
-                                               recv_scale, s));
-  cudaError_t e = moe::launch_layout(*prob, topk_idx, part_of, *lay, workspace, s);
+                                               recv_scale, t, s));
+  cudaError_t e = moe::launch_layout(*prob, topk_idx, part_of, *lay, workspace, s, t);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   return cuda_rc(moe::launch_dispatch(*prob, x, *lay, recv_x, recv_scale, s));
 }
@@ -111,14 +135,10 @@ size_t moe_expert_tiles_capacity(const moe_problem_t* prob, int32_t block_m) {
 }
 
 int moe_expert_tiles(const moe_problem_t* prob, const int32_t* part_of, const moe_layout_t* lay,
-                     int32_t block_m, int32_t* tile_first, int32_t* tile_expert,
-                     int32_t* tile_row, int32_t* tile_rows, moe_stream_t stream) {
-  if (!valid_problem(prob) || !valid_layout(prob, lay) || block_m < 1) return MOE_ERR_ARG;
-  if (!arr(part_of) || !arr(tile_first) || !arr(tile_expert) || !arr(tile_row) || !arr(tile_rows))
-    return MOE_ERR_ARG;
-  if (moe::expert_tiles_capacity(*prob, block_m) >= ((int64_t)1 << 31)) return MOE_ERR_ARG;
-  return cuda_rc(moe::launch_expert_tiles(*prob, part_of, *lay, block_m, tile_first, tile_expert,
-                                          tile_row, tile_rows,
+                     const moe_tiles_t* tiles, moe_stream_t stream) {
+  if (!valid_problem(prob) || !valid_layout(prob, lay) || !arr(part_of)) return MOE_ERR_ARG;
+  if (!valid_tiles(prob, tiles)) return MOE_ERR_ARG;
+  return cuda_rc(moe::launch_expert_tiles(*prob, part_of, *lay, *tiles,
                                           reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -129,21 +129,20 @@ int64_t expert_tiles_capacity(const moe_problem_t& p, int block_m) {
 }
 
 cudaError_t launch_expert_tiles(const moe_problem_t& p, const int32_t* part_of,
-                                const moe_layout_t& lay, int block_m, int32_t* tile_first,
-                                int32_t* tile_expert, int32_t* tile_row, int32_t* tile_rows,
+                                const moe_layout_t& lay, const moe_tiles_t& tiles,
                                 cudaStream_t stream) {
   TilesArgs a;
   a.G = p.G;
   a.E = p.E_part;
-  a.block_m = block_m;
-  a.max_tiles = expert_tiles_capacity(p, block_m);
+  a.block_m = tiles.block_m;
+  a.max_tiles = expert_tiles_capacity(p, tiles.block_m);
   a.part_of = part_of;
   a.expert_count = lay.expert_count;
   a.expert_offset = lay.expert_offset;
-  a.tile_first = tile_first;
-  a.tile_expert = tile_expert;
-  a.tile_row = tile_row;
-  a.tile_rows = tile_rows;
+  a.tile_first = tiles.tile_first;
+  a.tile_expert = tiles.tile_expert;
+  a.tile_row = tiles.tile_row;
+  a.tile_rows = tiles.tile_rows;
   a.status = lay.status;
   cudaError_t e = launch_pdl(expert_tiles_kernel, dim3(1), dim3(kXThreads), 0, stream, a);
   if (e != cudaSuccess) return e;

@@ -34,6 +34,9 @@
 //     waits for layout_count_kernel (programmatic dependent launch) -- then
 //     reduces the rows with batched 16-byte loads from L2 and ranks its tile.
 // In both, the tile's expert ids are cached in shared memory when they fit.
+// Asked for it, both also emit the grouped-GEMM tile metadata: one warp
+// scans the tiles per expert while the others rank, and every block writes
+// its share of the tiles at the end.
 #include <cooperative_groups.h>
 
 #include <algorithm>
@@ -49,6 +52,9 @@ namespace {
 
 constexpr int kLThreads = 512;
 constexpr int kLWarps = kLThreads / kWarp;
+// Register budget of the layout kernels: two blocks per SM, so that a rank
+// block that launches early (programmatic launch) fits beside a count block.
+constexpr int kLMinBlocks = 2;
 constexpr int kMaxCluster = 8;
 constexpr int kMaxTileItems = 16384;  // tile ids cached in shared memory (64 KB)
 // Compile-time tuning constants: batches of at most MOE_CLUSTER_ITEMS routed
@@ -97,6 +103,7 @@ struct LayoutArgs {
   int* disp_row;
   int* exp_to_disp;
   int* status;
+  TileOut tiles;  // grouped-GEMM tile metadata (tiles.block_m = 0: none)
 };
 
 struct Tile {
@@ -426,10 +433,33 @@ __device__ void rank_tile_items(const LayoutArgs& a, const Tile& tl, const Smem&
       [&](int i) { exp_row[i] = -1; });
 }
 
+// Tile metadata: one warp scans the tiles per expert in row order into
+// scanbuf (free once the offsets are final) with the experts in red (free
+// after the column sums) and the count in misc[3] ...
+__device__ void scan_tiles(const LayoutArgs& a, const Smem& S) {
+  const int n = tiles_scan_warp(S.pos, a.G, a.tiles.block_m, [&](int e) { return S.tot[e]; },
+                                S.scanbuf, S.red);
+  if (lane_id() == 0) S.misc[3] = n;
+}
+
+// ... and, after a block barrier, block b of nb writes its share of the tiles
+// (block 0 also each expert's first tile).
+__device__ void write_tiles(const LayoutArgs& a, const Smem& S, int b, int nb) {
+  const int n = S.misc[3];
+  if (b == 0) {
+    for (int e = threadIdx.x; e < a.G; e += kLThreads) a.tiles.tile_first[e] = S.scanbuf[S.pos[e]];
+    if (threadIdx.x == 0) a.tiles.tile_first[a.G] = n;
+  }
+  int i0, i1;
+  tiles_share(n, b, nb, i0, i1);
+  tiles_write(a.tiles, S.scanbuf, S.red, a.G, i0, i1, [&](int e) { return S.eoff[e]; },
+              [&](int e) { return S.tot[e]; });
+}
+
 // ---------------------------------------------------------------------------
 // schedule 1: one cluster of gridDim.x blocks
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kLThreads) layout_cluster_kernel(LayoutArgs a) {
+__global__ void __launch_bounds__(kLThreads, kLMinBlocks) layout_cluster_kernel(LayoutArgs a) {
   extern __shared__ __align__(16) int sm[];
   cg::cluster_group cluster = cg::this_cluster();
   const LayoutSmem P(a.G, a.E, a.W, a.key_cap);
@@ -464,15 +494,17 @@ __global__ void __launch_bounds__(kLThreads) layout_cluster_kernel(LayoutArgs a)
 
   const int R_exp = finish_offsets(a, S);
   if (r == 0) write_globals(a, S, R_exp);
+  if (a.tiles.block_m > 0 && warp_id() == 0) scan_tiles(a, S);
   if (a.dedup) rank_tile_parts(a, tl, S, ids);
-  rank_tile_items(a, tl, S, ids);
+  rank_tile_items(a, tl, S, ids);  // ends with a block barrier
+  if (a.tiles.block_m > 0) write_tiles(a, S, r, C);
   cluster.sync();  // no block leaves while another may still read its row
 }
 
 // ---------------------------------------------------------------------------
 // schedule 2: one tile per SM, two launches
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kLThreads) layout_count_kernel(LayoutArgs a) {
+__global__ void __launch_bounds__(kLThreads, kLMinBlocks) layout_count_kernel(LayoutArgs a) {
   extern __shared__ __align__(16) int sm[];
   const LayoutSmem P(a.G, a.E, a.W, a.key_cap);
   const Smem S(sm, P, a.G);
@@ -525,7 +557,7 @@ __device__ void column_sums(const int* src, int rows, int W, int b, int* red, in
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(kLThreads) layout_rank_kernel(LayoutArgs a) {
+__global__ void __launch_bounds__(kLThreads, kLMinBlocks) layout_rank_kernel(LayoutArgs a) {
   extern __shared__ __align__(16) int sm[];
   const LayoutSmem P(a.G, a.E, a.W, a.key_cap);
   const Smem S(sm, P, a.G);
@@ -544,8 +576,10 @@ __global__ void __launch_bounds__(kLThreads) layout_rank_kernel(LayoutArgs a) {
   column_sums(a.tile_rows, a.n_tiles, a.W, b, S.red, S.ctot, S.cpre);
   const int R_exp = finish_offsets(a, S);
   if (b == 0) write_globals(a, S, R_exp);
+  if (a.tiles.block_m > 0 && warp_id() == 0) scan_tiles(a, S);
   if (a.dedup) rank_tile_parts(a, tl, S, ids);
-  rank_tile_items(a, tl, S, ids);
+  rank_tile_items(a, tl, S, ids);  // ends with a block barrier
+  if (a.tiles.block_m > 0) write_tiles(a, S, b, a.n_tiles);
 }
 
 bool use_cluster(const moe_problem_t& p) { return (int64_t)p.M * p.topk <= kClusterItems; }
@@ -575,7 +609,7 @@ size_t layout_workspace_bytes(const moe_problem_t& p) {
 
 cudaError_t launch_layout(const moe_problem_t& p, const int32_t* topk_idx,
                           const int32_t* part_of, const moe_layout_t& lay,
-                          void* workspace, cudaStream_t stream) {
+                          void* workspace, cudaStream_t stream, const TileOut& tiles) {
   LayoutArgs a;
   a.M = p.M;
   a.G = p.G;
@@ -594,6 +628,7 @@ cudaError_t launch_layout(const moe_problem_t& p, const int32_t* topk_idx,
   a.disp_row = lay.disp_row;
   a.exp_to_disp = lay.exp_to_disp;
   a.status = lay.status;
+  a.tiles = tiles;
 
   if (use_cluster(p)) {
     const int items = p.M * p.topk;

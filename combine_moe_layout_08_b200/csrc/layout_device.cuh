@@ -62,4 +62,61 @@ __device__ __forceinline__ void expert_order_warp(const int* part_s, int G, int 
   __syncwarp();
 }
 
+// ---------------------------------------------------------------------------
+// grouped-GEMM tile metadata emitted by the layout kernels themselves
+// (DeepSpeed PR #8180, "Key points": per-tile -> group map from the offsets,
+// on the device): tiles of block_m rows that never straddle two experts,
+// numbered in row order.
+// ---------------------------------------------------------------------------
+struct TileOut {
+  int block_m;       // 0: no tiles requested
+  int* tile_first;   // [G + 1]
+  int* tile_expert;  // [cap]
+  int* tile_row;
+  int* tile_rows;
+};
+
+// One warp: tiles per expert in row order (pos[e] = the expert's position in
+// it, rows(e) = its rows) scanned into tscan[pos] = first tile, with
+// order[pos] = the expert; returns the number of tiles.  A layout's counts
+// sum to at most M * topk, so the total fits an int.
+template <class Rows>
+__device__ __forceinline__ int tiles_scan_warp(const int* pos, int G, int block_m, Rows rows,
+                                               int* tscan, int* order) {
+  for (int e = lane_id(); e < G; e += kWarp) {
+    const int c = rows(e);
+    tscan[pos[e]] = c > 0 ? (c - 1) / block_m + 1 : 0;
+    order[pos[e]] = e;
+  }
+  __syncwarp();
+  return warp_exclusive_scan(tscan, G);
+}
+
+// Tiles [i0, i1) (this block's share), all threads of the block: each finds
+// its expert by binary search in tscan (largest q with tscan[q] <= i) and
+// writes expert, first row (row_off(e) + j * block_m) and rows.
+template <class RowOff, class Rows>
+__device__ __forceinline__ void tiles_write(const TileOut& t, const int* tscan, const int* order,
+                                            int G, int i0, int i1, RowOff row_off, Rows rows) {
+  for (int i = i0 + (int)threadIdx.x; i < i1; i += (int)blockDim.x) {
+    int lo = 0, hi = G - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (tscan[mid] <= i) lo = mid; else hi = mid - 1;
+    }
+    const int e = order[lo];
+    const int j = i - tscan[lo];
+    t.tile_expert[i] = e;
+    t.tile_row[i] = row_off(e) + j * t.block_m;
+    t.tile_rows[i] = min(t.block_m, rows(e) - j * t.block_m);
+  }
+}
+
+// This block's share [i0, i1) of n tiles split over nb blocks.
+__device__ __forceinline__ void tiles_share(int n, int b, int nb, int& i0, int& i1) {
+  const int per = (n + nb - 1) / nb;
+  i0 = min(n, b * per);
+  i1 = min(n, i0 + per);
+}
+
 }  // namespace moe

@@ -22,7 +22,9 @@
 //        exp_row[t,k]  = expert_offset[e] + (pairs of e before t)
 //                        + (slots k' < k of t with the same expert)
 //        disp_row[t,p] = part_offset[p] + (tokens before t holding p)
-//   6. copies (bf16) or quantises and copies (fp8) its vectors to the rows.
+//   6. copies (bf16) or quantises and copies (fp8) its vectors to the rows;
+//   7. if asked, writes its share of the grouped-GEMM tile metadata (warp 1
+//      scanned the tiles per expert during step 5).
 // Every index is the one the tiled layout gives (stable (partition, expert,
 // token, slot) order, dedup rows in (partition, token) order), so results are
 // bit-identical to moe_layout followed by moe_dispatch.  Block (0, 0) writes
@@ -72,11 +74,12 @@ struct FusedArgs {
   int* disp_row;
   int* exp_to_disp;
   int* status;
+  TileOut tiles;  // grouped-GEMM tile metadata (tiles.block_m = 0: none)
 };
 
 // shared-memory plan in ints, every array 16-byte aligned
 struct FusedSmem {
-  int ids, part_s, hb, ha, pos, scan, kcnt, pb, pa, poff, prow, dst, nd, misc, total;
+  int ids, part_s, hb, ha, pos, scan, tscan, order, kcnt, pb, pa, poff, prow, dst, nd, misc, total;
   __host__ __device__ FusedSmem(int n_items, int G, int E) {
     int o = 0;
     ids = o; o += up4(n_items);   // every routing id
@@ -85,6 +88,8 @@ struct FusedSmem {
     ha = o; o += up4(G);          // ... from t0 on, then the expert's total
     pos = o; o += up4(G);         // expert -> position in (partition, id) order
     scan = o; o += up4(G);        // expert totals in that order -> exclusive scan
+    tscan = o; o += up4(G);       // tiles: first tile per expert in that order
+    order = o; o += up4(G);       // tiles: expert at each position of that order
     kcnt = o; o += up4(E + 1);    // scratch of the expert order
     pb = o; o += up4(E);          // dedup: tokens before the current token holding p
     pa = o; o += up4(E);          // ... from t0 on (without dedup: rows); then the total
@@ -92,7 +97,7 @@ struct FusedSmem {
     prow = o; o += up4(E);        // dedup: the current token's row per partition (-1: none)
     dst = o; o += kMaxChunk * kMaxDest;  // destination rows of each chunk token
     nd = o; o += kMaxChunk;              // ... and their number
-    misc = o; o += 4;             // [bad expert, bad placement, R_exp, unused]
+    misc = o; o += 4;             // [bad expert, bad placement, R_exp, number of tiles]
     total = o;
   }
 };
@@ -238,7 +243,13 @@ __global__ void __launch_bounds__(kFThreads, 1) layout_dispatch_kernel(FusedArgs
   __syncthreads();
 
   // 5. the chunk's rows, token by token (warp 0; hb and pb become running
-  // counters); the batch's counts and offsets (block (0, 0))
+  // counters); the tiles per expert (warp 1); the batch's counts and offsets
+  // (block (0, 0))
+  if (warp_id() == 1 && a.tiles.block_m > 0) {
+    const int n = tiles_scan_warp(pos, G, a.tiles.block_m, [&](int e) { return ha[e]; },
+                                  sm + P.tscan, sm + P.order);
+    if (lane_id() == 0) misc[3] = n;
+  }
   if (warp_id() == 0) {
     int* prow = sm + P.prow;
     const int lane = lane_id();
@@ -354,6 +365,19 @@ __global__ void __launch_bounds__(kFThreads, 1) layout_dispatch_kernel(FusedArgs
       }
     }
   }
+  // 7. this block's share of the tiles; block (0, 0): each expert's first tile
+  if (a.tiles.block_m > 0 && writer) {
+    const int* tscan = sm + P.tscan;
+    const int n = misc[3];
+    if (blockIdx.x == 0) {
+      for (int e = tid; e < G; e += kFThreads) a.tiles.tile_first[e] = tscan[pos[e]];
+      if (tid == 0) a.tiles.tile_first[G] = n;
+    }
+    int k0, k1;
+    tiles_share(n, blockIdx.x, gridDim.x, k0, k1);
+    tiles_write(a.tiles, tscan, sm + P.order, G, k0, k1, [&](int e) { return scan[pos[e]]; },
+                [&](int e) { return ha[e]; });
+  }
 }
 
 template <bool FP8, int U>
@@ -372,7 +396,7 @@ bool layout_dispatch_fused(const moe_problem_t& p) {
 cudaError_t launch_layout_dispatch(const moe_problem_t& p, const int32_t* topk_idx,
                                    const int32_t* part_of, const moe_layout_t& lay,
                                    const void* x, void* recv_x, float* recv_scale,
-                                   cudaStream_t stream) {
+                                   const TileOut& tiles, cudaStream_t stream) {
   FusedArgs a;
   a.M = p.M;
   a.G = p.G;
@@ -394,6 +418,7 @@ cudaError_t launch_layout_dispatch(const moe_problem_t& p, const int32_t* topk_i
   a.disp_row = lay.disp_row;
   a.exp_to_disp = lay.exp_to_disp;
   a.status = lay.status;
+  a.tiles = tiles;
 
   a.T = std::min(kMaxChunk, (p.M + kSMs - 1) / kSMs);
   const int blocks = (p.M + a.T - 1) / a.T;

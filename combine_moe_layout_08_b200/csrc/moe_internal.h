@@ -10,6 +10,10 @@
 
 #include "moe_layout.h"
 
+namespace moe {
+struct TileOut;  // layout_device.cuh
+}
+
 #ifndef MOE_USE_PDL
 #define MOE_USE_PDL 1  // programmatic dependent launch between the path's kernels
 #endif
@@ -51,9 +55,10 @@ int layout_tile_tokens(int M);
 int layout_num_tiles(int M);
 size_t layout_workspace_bytes(const moe_problem_t& p);
 
+// tiles: grouped-GEMM tile metadata to emit as well (tiles.block_m = 0: none)
 cudaError_t launch_layout(const moe_problem_t& p, const int32_t* topk_idx,
                           const int32_t* part_of, const moe_layout_t& lay,
-                          void* workspace, cudaStream_t stream);
+                          void* workspace, cudaStream_t stream, const TileOut& tiles);
 
 cudaError_t launch_dispatch(const moe_problem_t& p, const void* x,
                             const moe_layout_t& lay, void* recv_x,
@@ -64,13 +69,13 @@ bool layout_dispatch_fused(const moe_problem_t& p);
 cudaError_t launch_layout_dispatch(const moe_problem_t& p, const int32_t* topk_idx,
                                    const int32_t* part_of, const moe_layout_t& lay,
                                    const void* x, void* recv_x, float* recv_scale,
-                                   cudaStream_t stream);
+                                   const TileOut& tiles, cudaStream_t stream);
 
-// Grouped-GEMM tile metadata of a layout (entries per tile array: capacity).
+// Grouped-GEMM tile metadata of a finished layout, as its own kernel
+// (entries per tile array: capacity).
 int64_t expert_tiles_capacity(const moe_problem_t& p, int block_m);
 cudaError_t launch_expert_tiles(const moe_problem_t& p, const int32_t* part_of,
-                                const moe_layout_t& lay, int block_m, int32_t* tile_first,
-                                int32_t* tile_expert, int32_t* tile_row, int32_t* tile_rows,
+                                const moe_layout_t& lay, const moe_tiles_t& tiles,
                                 cudaStream_t stream);
 
 cudaError_t launch_combine_partial(const moe_problem_t& p, const void* y, const float* w,

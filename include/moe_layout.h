@@ -209,6 +209,32 @@ int moe_combine(const moe_problem_t *prob, const void *y,
                 moe_stream_t stream);
 
 /*
+ * Grouped-GEMM tile metadata of a layout (DeepSpeed PR #8180, "Key points":
+ * the per-tile -> group mapping of a grouped GEMM computed on the device
+ * from offs, so no device -> host copy).  Tiles hold block_m rows and never
+ * straddle two experts: expert e owns ceil(expert_count[e] / block_m)
+ * tiles, numbered in row order.  All arrays are device int32, caller-owned:
+ *   tile_first  [G+1]: first tile of expert e (also defined for experts
+ *               without rows); tile_first[G] = number of tiles
+ *   tile_expert [cap]: expert of tile i
+ *   tile_row    [cap]: first expert row of tile i
+ *   tile_rows   [cap]: rows of tile i, 1..block_m
+ * cap = moe_expert_tiles_capacity(prob, block_m) = ceil(M*topk/block_m) + G,
+ * the most a layout of this problem needs; entries past tile_first[G] are
+ * untouched.  Requests with block_m < 1, null or misaligned arrays, or a
+ * capacity of 2^31 entries or more are MOE_ERR_ARG.
+ */
+typedef struct {
+  int32_t block_m;
+  int32_t *tile_first;
+  int32_t *tile_expert;
+  int32_t *tile_row;
+  int32_t *tile_rows;
+} moe_tiles_t;
+
+size_t moe_expert_tiles_capacity(const moe_problem_t *prob, int32_t block_m);
+
+/*
  * Layout and dispatch in one call: the same results, bit for bit, as
  * moe_layout followed by moe_dispatch with the same arguments, and the same
  * argument rules and return codes as those two calls (workspace included).
@@ -216,44 +242,32 @@ int moe_combine(const moe_problem_t *prob, const void *y,
  * pairs by default), where both steps are bound by latency (Triton-
  * distributed issue #117, "Results (Latency in us)", M = 2..512) -- run as
  * ONE kernel in which every block rebuilds the small layout in shared
- * memory and dispatches its own token, with no inter-block wait; larger
- * batches run the two calls' kernels.  The workspace is left untouched by
- * the one-kernel schedule.
+ * memory and dispatches its own chunk of tokens, with no inter-block wait;
+ * larger batches run the two calls' kernels.  The workspace is left
+ * untouched by the one-kernel schedule.
+ * tiles (NULL: none) also fills the grouped-GEMM tile metadata, from inside
+ * the same kernels (no extra launch); the results equal moe_expert_tiles'.
  */
 int moe_layout_dispatch(const moe_problem_t *prob, const int32_t *topk_idx,
                         const int32_t *part_of, const moe_layout_t *lay,
                         void *workspace, size_t workspace_bytes, const void *x,
-                        void *recv_x, float *recv_scale, moe_stream_t stream);
+                        void *recv_x, float *recv_scale, const moe_tiles_t *tiles,
+                        moe_stream_t stream);
 
 /* 1 if moe_layout_dispatch takes the one-kernel schedule for `prob`, else 0
  * (also 0 for an invalid problem). */
 int moe_layout_dispatch_fused(const moe_problem_t *prob);
 
 /*
- * Grouped-GEMM tile metadata of a layout, computed on the device so that a
- * grouped GEMM over the expert rows needs no device -> host copy of the
- * offsets (DeepSpeed PR #8180, "Key points": per-tile -> group mapping
- * computed on device from offs).  Tiles hold block_m rows and never
- * straddle two experts: expert e owns ceil(expert_count[e] / block_m)
- * tiles, numbered in row order.  Call after moe_layout (same stream) with
- * the same part_of.
- *   tile_first  [G+1] int32: first tile of expert e (also defined for
- *               experts without rows); tile_first[G] = number of tiles
- *   tile_expert [cap] int32: expert of tile i
- *   tile_row    [cap] int32: first expert row of tile i
- *   tile_rows   [cap] int32: rows of tile i, 1..block_m
- * cap = moe_expert_tiles_capacity(prob, block_m) = ceil(M*topk/block_m) + G
- * entries, the most a layout of this problem needs; entries past
- * tile_first[G] are untouched.  Counts that cannot come from a layout of
- * this problem (more tiles than cap) write cap tiles and raise
- * MOE_STATUS_BAD_ROW.  MOE_ERR_ARG for block_m < 1, a capacity of 2^31 or
- * more, or null / misaligned arrays.
+ * The tile metadata (moe_tiles_t above) of a finished layout, as a kernel of
+ * its own: for callers of moe_layout or moe_layout_static.  Call after the
+ * layout on the same stream, with the same part_of.  Counts that cannot
+ * come from a layout of this problem (more tiles than the capacity) write
+ * only the capacity's tiles and raise MOE_STATUS_BAD_ROW.
  */
-size_t moe_expert_tiles_capacity(const moe_problem_t *prob, int32_t block_m);
 int moe_expert_tiles(const moe_problem_t *prob, const int32_t *part_of,
-                     const moe_layout_t *lay, int32_t block_m,
-                     int32_t *tile_first, int32_t *tile_expert,
-                     int32_t *tile_row, int32_t *tile_rows, moe_stream_t stream);
+                     const moe_layout_t *lay, const moe_tiles_t *tiles,
+                     moe_stream_t stream);
 
 /*
  * Two-level combine of a deduplicated dispatch (prob->dedup = 1, else

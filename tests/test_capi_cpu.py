@@ -150,9 +150,9 @@ def test_fused_schedule_query(L):
 def test_layout_dispatch_rejects_bad_arguments(L):
     lay = fake_layout()
     ws = L.moe_layout_workspace_size(ctypes.byref(P()))
-    call = lambda prob, idx=FAKE, po=FAKE, lay_=lay, w=FAKE, wb=ws, x=FAKE, r=FAKE, sc=None: \
+    call = lambda prob, idx=FAKE, po=FAKE, lay_=lay, w=FAKE, wb=ws, x=FAKE, r=FAKE, sc=None, t=None: \
         L.moe_layout_dispatch(ctypes.byref(prob), idx, po, ctypes.byref(lay_) if lay_ else None,
-                              w, wb, x, r, sc, None)
+                              w, wb, x, r, sc, ctypes.byref(t) if t else None, None)
     assert call(P(N=12)) == 1
     assert call(P(), idx=FAKE + 2) == 1
     assert call(P(), po=None) == 1
@@ -162,6 +162,10 @@ def test_layout_dispatch_rejects_bad_arguments(L):
     assert call(P(dedup=1), lay_=fake_layout(exp_to_disp=None)) == 1
     assert call(P(), wb=ws - 1) == 2
     assert call(P(), w=FAKE + 8) == 2
+    # an invalid tile request
+    assert call(P(), t=_lib.TilesStruct(0, FAKE, FAKE, FAKE, FAKE)) == 1
+    assert call(P(), t=_lib.TilesStruct(128, FAKE, None, FAKE, FAKE)) == 1
+    assert call(P(), t=_lib.TilesStruct(128, FAKE, FAKE, FAKE + 2, FAKE)) == 1
 
 
 def test_expert_tiles_capacity(L):
@@ -176,12 +180,14 @@ def test_expert_tiles_capacity(L):
 def test_expert_tiles_rejects_bad_arguments(L):
     lay = fake_layout()
     p = ctypes.byref(P())
+    T = lambda bm, *arrs: ctypes.byref(_lib.TilesStruct(bm, *arrs))
     ok = (FAKE, FAKE + 64, FAKE + 128, FAKE + 192)
-    assert L.moe_expert_tiles(p, FAKE, ctypes.byref(lay), 0, *ok, None) == 1
-    assert L.moe_expert_tiles(p, None, ctypes.byref(lay), 64, *ok, None) == 1
-    assert L.moe_expert_tiles(p, FAKE, None, 64, *ok, None) == 1
-    assert L.moe_expert_tiles(p, FAKE, ctypes.byref(lay), 64, FAKE, FAKE + 2, FAKE, FAKE, None) == 1
-    assert L.moe_expert_tiles(p, FAKE, ctypes.byref(lay), 64, FAKE, FAKE, FAKE, None, None) == 1
+    assert L.moe_expert_tiles(p, FAKE, ctypes.byref(lay), T(0, *ok), None) == 1
+    assert L.moe_expert_tiles(p, None, ctypes.byref(lay), T(64, *ok), None) == 1
+    assert L.moe_expert_tiles(p, FAKE, None, T(64, *ok), None) == 1
+    assert L.moe_expert_tiles(p, FAKE, ctypes.byref(lay), T(64, FAKE, FAKE + 2, FAKE, FAKE), None) == 1
+    assert L.moe_expert_tiles(p, FAKE, ctypes.byref(lay), T(64, FAKE, FAKE, FAKE, None), None) == 1
+    assert L.moe_expert_tiles(p, FAKE, ctypes.byref(lay), None, None) == 1
 
 
 def test_python_binding_fails_loudly_without_library(monkeypatch, tmp_path):

@@ -93,3 +93,30 @@ def test_empty_batch():
     torch.cuda.synchronize()
     assert np.all(t.tile_first.cpu().numpy() == 0)
     assert np.all(t.tile_expert.cpu().numpy() == POISON_I32)
+
+
+# tiles emitted by moe_layout_dispatch from inside each layout schedule
+@pytest.mark.parametrize("M,G,topk,E,dedup,fp8", [
+    (128, 256, 8, 8, False, False),    # one kernel for layout + dispatch
+    (900, 256, 8, 8, True, False),     # one-cluster layout (7200 pairs)
+    (4096, 256, 8, 8, False, True),    # two-launch tiled layout
+    (3000, 1024, 32, 64, True, False),  # largest G / topk / E_part, tiled
+])
+@pytest.mark.parametrize("block_m", [1, 128])
+def test_tiles_from_layout_dispatch(M, G, topk, E, dedup, fp8, block_m):
+    from gpu_harness import compare_dispatch_rows, compare_layout, untouched_rows_ok
+    w = W.Workload("tiles-ld", M=M, N=128, G=G, topk=topk, E_part=E, routing="zipf",
+                   placement="contiguous", dedup=dedup, fp8=fp8, zipf_s=1.2, seed=M + block_m)
+    prob = problem_of(w)
+    d = W.make_inputs(w, device=DEV, with_y=False)
+    po = np.random.default_rng(M).permutation(d["part_of"]).astype(np.int32)
+    b = poisoned_buffers(prob, DEV)
+    t, _ = _tiles(prob, block_m)
+    b.tiles = t
+    b.layout_dispatch_(to_dev(d["topk_idx"]), to_dev(po), d["x"], block_m=block_m)
+    torch.cuda.synchronize()
+    lay = oracle.layout(d["topk_idx"], po, G, E, dedup)
+    compare_layout(b, lay, prob)
+    compare_dispatch_rows(b, prob, oracle.bf16_bits(d["x"]), lay["disp_token"])
+    untouched_rows_ok(b, lay["R_disp"])
+    _compare(t, oracle.expert_tiles(lay["expert_count"], lay["expert_offset"], block_m))
