@@ -2,15 +2,17 @@
 """Benchmark of the MoE dispatch / combine path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME]
+                    [--workload NAME] [--schedule auto|separate] [--tiles BM]
+                    [--combine one-level|two-level] [--latency-sweep]
 
 One step = one pass of the whole path over one batch: routing layout ->
 dispatch permute -> combine (libmoe_layout.so, through its C ABI), on the
 M = 4096, N = 7168, G = 256, topk = 8, E_part = 8, Zipf(1.1) workload by
 default.  Inputs are resident in HBM when the timed region starts.  Each
-step is one CUDA-graph replay whose events bracket its kernels on the
-device; L2 is flushed between steps (256 MiB written, then 256 MiB read,
-untimed).
+step is one CUDA-graph replay with events at its two ends on the device;
+a second graph of the same step with events between its parts gives the
+per-kernel breakdown.  L2 is flushed between steps (256 MiB written, then
+256 MiB read, untimed).
 
 Printed (rank 0, one JSON line): value = algorithmic HBM bytes of the whole
 path per second (GB/s) over all ranks; tokens/s; per-kernel times; the
@@ -397,6 +399,7 @@ def run_ours(args, w):
     if world > 1:
         dist.barrier()
     total_ms = float(np.sum(step_ms))
+    step_us = np.array(step_ms) * 1e3
     # per-kernel breakdown (untimed for the headline; same flush, same inputs)
     for _ in range(3):
         parts_step()
@@ -426,6 +429,9 @@ def run_ours(args, w):
             "metric": METRIC, "value": round(all_bytes / (max_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(max_ms / args.steps, 5), "higher_is_better": True,
+            "step_us": {"mean": round(float(step_us.mean()), 2),
+                        "median": round(float(np.median(step_us)), 2),
+                        "best": round(float(step_us.min()), 2), "note": "rank 0"},
             "scaling": "weak", "vs_baseline": None, "dtype": "f8e4m3+bf16" if w.fp8 else "bf16",
             "data": "synthetic",
             "tokens_per_s": round(all_tokens / (max_ms * 1e-3), 1),
@@ -464,6 +470,7 @@ def run_ours(args, w):
         dist.destroy_process_group()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wr, buf, idx_h, po_h, g_h, x, y)
+        line["cpu_baseline_all_cores"] = cpu_baseline_parallel(wr, idx_h, po_h, g_h, x, y)
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
@@ -536,9 +543,76 @@ def cpu_baseline(w, buf, idx_h, po_h, g_h, x, y, budget_s=10.0):
     mean = sum(times) / len(times)
     what = f"full {w.name} problem (M={w.M})" if m == w.M else \
         f"first {m} of the {w.M} tokens of {w.name}"
+    model, cores = host_cpu()
     return {"value": round(b / mean / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "tokens_per_s": round(m / mean, 1),
+            "tokens_per_s": round(m / mean, 1), "cpu": model, "host_cores": cores,
             "sample": f"{what}, {len(times)} oracle passes, {sum(times):.1f} s, single thread"}
+
+
+def host_cpu():
+    """Model name and usable cores of this host."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return model, len(os.sched_getaffinity(0))
+
+
+def _oracle_shard(job):
+    """Worker of cpu_baseline_parallel (its own process): the oracle as it
+    stands on one shard of tokens, as a problem of its own, repeated for
+    about ``budget`` seconds; returns (seconds, passes, algorithmic bytes)."""
+    import oracle
+    fields, idx, po, gates, xb, yb, budget = job
+    w = W.Workload(**fields)
+    times, lay = [], None
+    while sum(times) < budget and len(times) < 50:
+        t, lay = oracle_step_seconds(w, idx, po, gates, xb, yb)
+        times.append(t)
+    return sum(times), len(times), sum(algorithmic_bytes(w, lay["R_exp"], lay["R_disp"]).values())
+
+
+def cpu_baseline_parallel(w, idx_h, po_h, g_h, x, y, budget_s=10.0):
+    """The same oracle on every usable host core: one spawned process per
+    core, each on its own shard of the first tokens of the batch (the shards
+    are independent problems, like data-parallel replicas).  Throughput =
+    the shards' bytes / the slowest shard's time.  Returns the reason
+    instead if the pool cannot run here."""
+    import dataclasses
+    import multiprocessing as mp
+
+    import oracle
+    model, cores = host_cpu()
+    P = max(1, min(cores, 64))
+    per = max(1, min(w.M // P, 1024))
+    m = per * P
+    fields = {f.name: getattr(w, f.name) for f in dataclasses.fields(w)}
+    fields["M"] = per
+    jobs = []
+    for i in range(P):
+        t0, t1 = i * per, (i + 1) * per
+        jobs.append((fields, idx_h[t0:t1], po_h, g_h[t0:t1], oracle.bf16_bits(x[t0:t1]),
+                     oracle.bf16_bits(y[t0 * w.topk:t1 * w.topk]), budget_s))
+    # a broken worker (e.g. one that cannot start) raises here instead of
+    # hanging, and every result is bounded in time
+    from concurrent.futures import ProcessPoolExecutor
+    try:
+        with ProcessPoolExecutor(P, mp_context=mp.get_context("spawn")) as ex:
+            futs = [ex.submit(_oracle_shard, j) for j in jobs]
+            res = [f.result(timeout=6 * budget_s + 300) for f in futs]
+    except Exception as e:  # a host that cannot run the workers: say so in the line
+        return {"unavailable": f"{type(e).__name__}: {e}"}
+    slowest = max(r[0] / r[1] for r in res)         # seconds per pass of the slowest shard
+    b = sum(r[2] for r in res)
+    return {"value": round(b / slowest / 1e9, 4), "unit": "GB/s", "cores": P, "kind": "oracle",
+            "tokens_per_s": round(m / slowest, 1), "cpu": model, "host_cores": cores,
+            "sample": f"first {m} tokens of {w.name} in {P} shards of {per} (one process "
+                      f"per core, each about {budget_s:.0f} s)"}
 
 
 def run_latency_sweep(args):
