@@ -27,77 +27,11 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
   return v;
 }
 
-// Read-only gather of a row that another pass of the kernel does not revisit.
-__device__ __forceinline__ uint4 ld_nc_v4_evict_first(const void* p) {
-  uint4 v;
-  asm("ld.global.nc.L1::no_allocate.L2::evict_first.v4.u32 {%0, %1, %2, %3}, [%4];"
-      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-      : "l"(p));
-  return v;
-}
-
 // Store that does not allocate in L1.
 __device__ __forceinline__ void st_v4(void* p, const uint4& v) {
   asm volatile("st.global.L1::no_allocate.v4.u32 [%0], {%1, %2, %3, %4};"
                :
                : "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-               : "memory");
-}
-
-// Streaming store (evict-first in L2): output rows nobody re-reads soon.
-__device__ __forceinline__ void st_cs_v4(void* p, const uint4& v) {
-  asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};"
-               :
-               : "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-               : "memory");
-}
-
-// W 32-bit words moved as one vector: W = 4 (16 bytes) or W = 8 (32 bytes,
-// 256-bit loads and stores on sm_100a; addresses 32-byte aligned).
-template <int W>
-struct Vec {
-  uint32_t w[W];
-};
-
-template <int W>
-__device__ __forceinline__ Vec<W> ld_nc(const void* p);
-
-template <>
-__device__ __forceinline__ Vec<4> ld_nc<4>(const void* p) {
-  Vec<4> v;
-  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-      : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3])
-      : "l"(p));
-  return v;
-}
-
-template <>
-__device__ __forceinline__ Vec<8> ld_nc<8>(const void* p) {
-  Vec<8> v;
-  asm("ld.global.nc.L1::no_allocate.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-      : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3]), "=r"(v.w[4]), "=r"(v.w[5]),
-        "=r"(v.w[6]), "=r"(v.w[7])
-      : "l"(p));
-  return v;
-}
-
-template <int W>
-__device__ __forceinline__ void st_na(void* p, const Vec<W>& v);
-
-template <>
-__device__ __forceinline__ void st_na<4>(void* p, const Vec<4>& v) {
-  asm volatile("st.global.L1::no_allocate.v4.u32 [%0], {%1, %2, %3, %4};"
-               :
-               : "l"(p), "r"(v.w[0]), "r"(v.w[1]), "r"(v.w[2]), "r"(v.w[3])
-               : "memory");
-}
-
-template <>
-__device__ __forceinline__ void st_na<8>(void* p, const Vec<8>& v) {
-  asm volatile("st.global.L1::no_allocate.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
-               :
-               : "l"(p), "r"(v.w[0]), "r"(v.w[1]), "r"(v.w[2]), "r"(v.w[3]), "r"(v.w[4]),
-                 "r"(v.w[5]), "r"(v.w[6]), "r"(v.w[7])
                : "memory");
 }
 
