@@ -11,8 +11,8 @@ import torch
 import combine_moe_layout_08_b200 as moe
 import oracle
 import workloads as W
-from gpu_harness import (compare_dispatch_rows, compare_layout, poisoned_buffers, problem_of, to_dev,
-                         untouched_rows_ok)
+from gpu_harness import (POISON_I32, compare_dispatch_rows, compare_layout, poisoned_buffers,
+                         problem_of, to_dev, untouched_rows_ok)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -124,3 +124,43 @@ def test_repeat_and_graph_capture():
         g.replay()
     torch.cuda.synchronize()
     assert torch.equal(b.recv_x, first[0]) and torch.equal(b.layout.exp_row, first[1])
+
+
+@pytest.mark.parametrize("dedup,fp8", [(False, False), (True, True)])
+def test_empty_batch(dedup, fp8):
+    """M = 0: counts and offsets all zero, status 0, no row written, no tiles."""
+    prob = moe.MoEProblem(0, 256, 16, 4, 4, dedup, fp8)
+    assert not moe.moe_layout_dispatch_fused(prob)
+    b = poisoned_buffers(prob, DEV)
+    b.tiles = moe.alloc_expert_tiles(prob, 64, DEV)
+    for t in (b.tiles.tile_first, b.tiles.tile_expert, b.tiles.tile_row, b.tiles.tile_rows):
+        t.fill_(POISON_I32)
+    po = torch.arange(16, dtype=torch.int32, device=DEV) % 4
+    x = torch.zeros((1, 256), dtype=torch.bfloat16, device=DEV)
+    b.layout_dispatch_(torch.zeros(1, dtype=torch.int32, device=DEV), po, x, block_m=64)
+    torch.cuda.synchronize()
+    assert int(b.layout.status.item()) == 0
+    for t in (b.layout.expert_count, b.layout.expert_offset, b.layout.part_count,
+              b.layout.part_offset, b.tiles.tile_first):
+        assert bool((t == 0).all())
+    assert bool((b.tiles.tile_expert == POISON_I32).all())
+
+
+def test_binding_rejects_bad_tensors():
+    w = W.get("decode-M128-uniform")
+    prob = problem_of(w)
+    d = W.make_inputs(w, device=DEV, with_y=False)
+    b = moe.MoEBuffers(prob, DEV)
+    idx, po = to_dev(d["topk_idx"]), to_dev(d["part_of"])
+    with pytest.raises(TypeError):
+        b.layout_dispatch_(idx.long(), po, d["x"])
+    with pytest.raises(ValueError):
+        b.layout_dispatch_(idx, po, d["x"][:, ::2])            # not contiguous
+    with pytest.raises(ValueError):
+        b.layout_dispatch_(idx, po, d["x"][:64])               # too few rows
+    with pytest.raises(ValueError):
+        moe.alloc_expert_tiles(prob, 0, DEV)                   # block_m < 1
+    t = moe.alloc_expert_tiles(prob, 128, DEV)
+    t.tile_row = t.tile_row[:10]
+    with pytest.raises(ValueError):
+        moe.moe_layout_dispatch(prob, idx, po, b.layout, b.workspace, d["x"], b.recv_x, tiles=t)
