@@ -14,7 +14,9 @@
  * Conventions shared by every entry point
  *   - Every pointer argument except `prob` and `lay` (host structs) is a
  *     DEVICE pointer, owned and allocated by the caller; nothing is allocated,
- *     freed or kept by the library.  Device buffers must be 16-byte aligned.
+ *     freed or kept by the library.  Row buffers (x, y, recv_x, recv_scale,
+ *     out, z) and the workspace must be 16-byte aligned, int32 arrays 4-byte
+ *     aligned.
  *   - Calls are asynchronous on `stream` (NULL = legacy default stream) and
  *     never synchronise with the host or copy device data back to it.  Two
  *     calls on different streams that share an output race.
@@ -106,8 +108,10 @@ typedef struct moe_problem {
  *   exp_to_disp   [M*topk]   dedup only: dispatch row holding the token of
  *                            each expert row (first R_exp used); may be NULL
  *                            without dedup.
- *   status        [1]        MOE_STATUS_* bits; written by moe_layout,
- *                            OR-ed into by moe_dispatch / moe_combine.
+ *   status        [1]        MOE_STATUS_* bits; written by the layout
+ *                            (moe_layout, moe_layout_static,
+ *                            moe_layout_dispatch), OR-ed into by the calls
+ *                            that read the layout afterwards.
  * Entries beyond R_exp / R_disp are left untouched.
  */
 typedef struct moe_layout {
