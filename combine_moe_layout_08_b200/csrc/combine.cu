@@ -8,8 +8,8 @@
 //
 // One block of 128 threads per (token, column slice).  The token's slot rows
 // and gates are read once into shared memory.  A thread owns U 16-byte
-// vectors and gathers KG slots of all of them before the first accumulation
-// (KG * U = 8 loads in flight per thread for any topk: few slots -> more
+// vectors and gathers KG slots of all of them before accumulating them in
+// order (KG * U = 4 to 8 loads in flight per thread: few slots -> more
 // columns per thread), so the fixed order costs no memory parallelism.
 #include <algorithm>
 
@@ -124,8 +124,11 @@ cudaError_t launch_combine(const moe_problem_t& p, const void* y, const float* w
   a.topk = p.topk;
   a.cap = p.M * p.topk;
   a.status = lay.status;
-  // KG slots gathered per batch x U vectors per thread = 8 loads in flight
-  if (p.topk >= 5) return launch<8, 1>(a, p.M, stream);
+  // KG slots gathered per batch x U vectors per thread.  Measured on B200
+  // (combine us at topk 8, M4096 / M8192 / M65536): KG = 4 beats 8, 2 and 1
+  // (90.2 / 170.3 / 1290 against 90.6 / 172.5 / 1307 for 8, 91.3 / 174.0 /
+  // 1316 for 2); at topk 2, U = 4 beats 2 and 1.
+  if (p.topk >= 5) return launch<4, 1>(a, p.M, stream);
   if (p.topk >= 3) return launch<4, 2>(a, p.M, stream);
   if (p.topk == 2) return launch<2, 4>(a, p.M, stream);
   return launch<1, 8>(a, p.M, stream);
