@@ -331,7 +331,12 @@ def moe_combine_reduce(prob: MoEProblem, z: torch.Tensor, lay: MoELayout, out: t
 
 class MoEBuffers:
     """Caller-side device buffers of one problem at worst-case capacity, and
-    the three calls of one pass over them (layout -> dispatch -> combine)."""
+    the calls of one pass over them (layout -> dispatch -> combine).
+
+    Each call checks the caller's tensors; the buffers of this object are
+    checked again only when one of them has been replaced since its last
+    check (a few microseconds of host time per call, which matters in
+    decode loops)."""
 
     def __init__(self, prob: MoEProblem, device="cuda"):
         self.prob = prob
@@ -347,33 +352,116 @@ class MoEBuffers:
             self.recv_x = torch.empty((cap, prob.N), dtype=torch.bfloat16, device=self.device)
             self.recv_scale = None
         self.out = torch.empty((max(prob.M, 1), prob.N), dtype=torch.bfloat16, device=self.device)
+        self.device = self.out.device          # with its index ("cuda" -> "cuda:0")
+        self.z = None
+        self.tiles = None
+        self._lib = _lib.load()
+        self._ps = prob.struct()
+        self._ts = None
+        self._seen = {}
+
+    def _run(self, name, rc):
+        if rc:
+            raise MoEError(name, rc)
+
+    def _inputs(self, stream, *checks):
+        for t, name, dtype, numel in checks:
+            _check(t, name, dtype, numel, self.device)
+        return _stream(checks[0][0], stream)
+
+    def _own(self, name, dtype, numel):
+        """Device pointer of this object's buffer ``name``, checked again
+        whenever the tensor there is not the one checked last."""
+        t = getattr(self, name)
+        if t is None:
+            return None
+        key = (id(t), t.data_ptr())
+        if self._seen.get(name) != key:
+            _check(t, name, dtype, numel, self.device)
+            self._seen[name] = key
+        return key[1]
+
+    @staticmethod
+    def _key(obj):
+        """Identity and address of every tensor field of a dataclass (a
+        replaced array changes the first, a moved one the second)."""
+        return tuple(None if t is None else (id(t), t.data_ptr())
+                     for t in (getattr(obj, f.name) for f in dataclasses.fields(obj))
+                     if t is None or isinstance(t, torch.Tensor))
+
+    def _lay(self):
+        """The layout struct, its arrays checked again when any changed."""
+        key = self._key(self.layout)
+        if self._seen.get("layout") != key:
+            _check_layout(self.prob, self.layout, self.device)
+            self._seen["layout"] = key
+        return self.layout.struct()
+
+    def _recv(self):
+        p = self.prob
+        rx = self._own("recv_x", torch.uint8 if p.fp8 else torch.bfloat16, p.capacity * p.N)
+        rs = self._own("recv_scale", torch.float32, p.capacity * (p.N // 128)) if p.fp8 else None
+        return rx, rs
 
     def layout_(self, topk_idx, part_of, stream=None):
-        moe_layout(self.prob, topk_idx, part_of, self.layout, self.workspace, stream)
+        p = self.prob
+        st = self._inputs(stream, (topk_idx, "topk_idx", torch.int32, p.M * p.topk),
+                          (part_of, "part_of", torch.int32, p.G))
+        ws = self._own("workspace", torch.uint8, None)
+        self._run("moe_layout", self._lib.moe_layout(
+            ctypes.byref(self._ps), topk_idx.data_ptr(), part_of.data_ptr(),
+            ctypes.byref(self._lay()), ws, self.workspace.numel(), st))
 
     def dispatch_(self, x, stream=None):
-        moe_dispatch(self.prob, x, self.layout, self.recv_x, self.recv_scale, stream)
+        p = self.prob
+        st = self._inputs(stream, (x, "x", torch.bfloat16, p.M * p.N))
+        rx, rs = self._recv()
+        self._run("moe_dispatch", self._lib.moe_dispatch(
+            ctypes.byref(self._ps), x.data_ptr(), ctypes.byref(self._lay()), rx, rs, st))
 
     def _tiles_for(self, block_m):
-        t = getattr(self, "tiles", None)
+        t = self.tiles
         if t is None or t.block_m != block_m:
             self.tiles = t = alloc_expert_tiles(self.prob, block_m, self.device)
+            self._ts = t.struct()
+        else:
+            key = self._key(t)
+            if self._seen.get("tiles") != key:     # arrays set by the caller
+                _check_tiles(self.prob, t, self.device)
+                self._seen["tiles"] = key
+            self._ts = t.struct()
         return t
 
     def layout_dispatch_(self, topk_idx, part_of, x, stream=None, block_m=None):
         """moe_layout_dispatch; ``block_m`` also fills ``self.tiles`` from the
         same kernels."""
-        moe_layout_dispatch(self.prob, topk_idx, part_of, self.layout, self.workspace, x,
-                            self.recv_x, self.recv_scale,
-                            self._tiles_for(block_m) if block_m else None, stream)
+        p = self.prob
+        st = self._inputs(stream, (x, "x", torch.bfloat16, p.M * p.N),
+                          (topk_idx, "topk_idx", torch.int32, p.M * p.topk),
+                          (part_of, "part_of", torch.int32, p.G))
+        ts = None
+        if block_m:
+            self._tiles_for(block_m)
+            ts = ctypes.byref(self._ts)
+        rx, rs = self._recv()
+        ws = self._own("workspace", torch.uint8, None)
+        self._run("moe_layout_dispatch", self._lib.moe_layout_dispatch(
+            ctypes.byref(self._ps), topk_idx.data_ptr(), part_of.data_ptr(), ctypes.byref(self._lay()),
+            ws, self.workspace.numel(), x.data_ptr(), rx, rs, ts, st))
 
     def combine_(self, y, topk_weights, stream=None):
-        moe_combine(self.prob, y, topk_weights, self.layout, self.out, stream)
+        p = self.prob
+        st = self._inputs(stream, (y, "y", torch.bfloat16, p.capacity * p.N),
+                          (topk_weights, "topk_weights", torch.float32, p.M * p.topk))
+        out = self._own("out", torch.bfloat16, p.M * p.N)
+        self._run("moe_combine", self._lib.moe_combine(
+            ctypes.byref(self._ps), y.data_ptr(), topk_weights.data_ptr(), ctypes.byref(self._lay()),
+            out, st))
 
     def combine_two_level_(self, y, topk_weights, stream=None):
         """Two-level combine through the dispatch-row buffer ``self.z``
         (allocated on first use)."""
-        if getattr(self, "z", None) is None:
+        if self.z is None:
             self.z = torch.empty((max(self.prob.capacity, 1), self.prob.N), dtype=torch.bfloat16,
                                  device=self.device)
         moe_combine_partial(self.prob, y, topk_weights, self.layout, self.z, stream)

@@ -164,3 +164,25 @@ def test_binding_rejects_bad_tensors():
     t.tile_row = t.tile_row[:10]
     with pytest.raises(ValueError):
         moe.moe_layout_dispatch(prob, idx, po, b.layout, b.workspace, d["x"], b.recv_x, tiles=t)
+
+
+def test_replaced_buffers_are_checked_again():
+    """MoEBuffers checks its own buffers once, and again after one is replaced."""
+    w = W.get("decode-M128-uniform")
+    prob = problem_of(w)
+    d = W.make_inputs(w, device=DEV)
+    idx, po, g = to_dev(d["topk_idx"]), to_dev(d["part_of"]), to_dev(d["topk_weights"])
+    b = moe.MoEBuffers(prob, DEV)
+    b.layout_dispatch_(idx, po, d["x"])
+    b.recv_x = b.recv_x[:10]                                   # too few rows
+    with pytest.raises(ValueError):
+        b.layout_dispatch_(idx, po, d["x"])
+    b = moe.MoEBuffers(prob, DEV)
+    b.layout_dispatch_(idx, po, d["x"])
+    b.layout.exp_row = b.layout.exp_row[:5]                    # too short
+    with pytest.raises(ValueError):
+        b.combine_(d["y"], g)
+    b = moe.MoEBuffers(prob, DEV)
+    b.out = b.out.float()                                      # wrong dtype
+    with pytest.raises(TypeError):
+        b.step(idx, po, d["x"], d["y"], g)
