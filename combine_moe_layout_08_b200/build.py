@@ -10,6 +10,7 @@ spills, shared memory) goes to ``_build/ptxas.log``.
 """
 from __future__ import annotations
 
+import concurrent.futures
 import glob
 import os
 import shutil
@@ -60,12 +61,18 @@ def build(force: bool = False, verbose: bool = False, defines=(), out: str = Non
     nvcc = _nvcc()
     bdir = BUILD if out is None else os.path.join(os.path.dirname(os.path.abspath(out)), "_obj")
     os.makedirs(bdir, exist_ok=True)
-    objs, log = [], []
-    for src in sources():
+    def compile_one(src):
         obj = os.path.join(bdir, os.path.basename(src) + ".o")
         cmd = [nvcc, *ARCH, *NVFLAGS, *[f"-D{d}" for d in defines], "-I", INCLUDE, "-I", CSRC,
                "-c", src, "-o", obj]
-        res = subprocess.run(cmd, capture_output=True, text=True)
+        return src, obj, cmd, subprocess.run(cmd, capture_output=True, text=True)
+
+    # one nvcc process per translation unit, in parallel
+    srcs = sources()
+    with concurrent.futures.ThreadPoolExecutor(max_workers=min(len(srcs), os.cpu_count() or 1)) as ex:
+        results = list(ex.map(compile_one, srcs))
+    objs, log = [], []
+    for src, obj, cmd, res in results:
         log.append(f"$ {' '.join(cmd)}\n{res.stdout}{res.stderr}")
         if res.returncode != 0:
             raise RuntimeError(f"nvcc failed on {src}:\n{res.stderr}")

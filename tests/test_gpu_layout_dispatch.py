@@ -186,3 +186,25 @@ def test_replaced_buffers_are_checked_again():
     b.out = b.out.float()                                      # wrong dtype
     with pytest.raises(TypeError):
         b.step(idx, po, d["x"], d["y"], g)
+
+
+@pytest.mark.parametrize("M,topk,dedup", [(128, 8, False),     # one kernel
+                                          (1000, 8, True),     # one-cluster layout
+                                          (4096, 8, False)])   # two-launch tiled layout
+def test_routing_ids_not_16_byte_aligned(M, topk, dedup):
+    """topk_idx starting 4 bytes past a 16-byte boundary takes the scalar
+    staging path of every layout schedule; the results are the same."""
+    w = W.Workload("ld-unaligned", M=M, N=64, G=256, topk=topk, E_part=8, routing="zipf",
+                   placement="contiguous", dedup=dedup, zipf_s=1.1, seed=M)
+    d = W.make_inputs(w, device=DEV, with_y=False)
+    flat = torch.empty(M * topk + 1, dtype=torch.int32, device=DEV)
+    idx = flat[1:].view(M, topk)
+    idx.copy_(to_dev(d["topk_idx"]))
+    assert idx.data_ptr() % 16 == 4
+    prob = problem_of(w)
+    b = poisoned_buffers(prob, DEV)
+    b.layout_dispatch_(idx, to_dev(d["part_of"]), d["x"])
+    torch.cuda.synchronize()
+    ref = oracle.layout(d["topk_idx"], d["part_of"], w.G, w.E_part, w.dedup)
+    compare_layout(b, ref, prob)
+    compare_dispatch_rows(b, prob, oracle.bf16_bits(d["x"]), ref["disp_token"])
