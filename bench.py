@@ -32,6 +32,7 @@ import datetime
 import hashlib
 import json
 import os
+import re
 import statistics
 import sys
 import threading
@@ -80,20 +81,31 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def source_digest(names) -> str:
+    """First 16 hex digits of the SHA-256 of the kernel sources ``names``
+    (files of the library's csrc/) with comments and whitespace removed, so
+    that only a change of the code itself changes it."""
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "combine_moe_layout_08_b200", "csrc", n)) as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        h.update(re.sub(r"\s+", "", text).encode())
+    return h.hexdigest()[:16]
+
+
 def traffic_record(kernel: str, workload: str):
     """DRAM bytes per launch from a committed ncu summary, if the kernel's
-    source is unchanged since the capture (else None)."""
+    code is unchanged since the capture (else None)."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         with open(p) as f:
             rec = json.load(f)[f"{kernel}@{workload}"]
-        h = hashlib.sha256()
-        for s in rec["sources"]:
-            with open(os.path.join(ROOT, "combine_moe_layout_08_b200", "csrc", s), "rb") as f:
-                h.update(f.read())
+        ok = source_digest(rec["sources"]) == rec["source_sha256_16"]
     except Exception:
         return None
-    return float(rec["bytes_per_launch"]) if h.hexdigest()[:16] == rec["source_sha256_16"] else None
+    return float(rec["bytes_per_launch"]) if ok else None
 
 
 # ---------------------------------------------------------------------------

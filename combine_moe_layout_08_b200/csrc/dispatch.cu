@@ -5,8 +5,12 @@
 // (WITH_SCALE); here the destinations are partitions of one receive buffer
 // in this GPU's HBM.
 //
-// bf16: 16-byte vector loads (non-coherent, no L1 allocation) of the whole
-// row segment into registers, then 16-byte stores to each destination.
+// One block of 128 threads per (token, column slice): a fan-out dispatch (no
+// dedup, topk >= 4) cuts each row into slices of one 16-byte vector per
+// thread; otherwise a block takes the whole row (up to 8 vectors per thread).
+//
+// bf16: 16-byte vector loads (non-coherent, no L1 allocation) of the block's
+// row slice into registers, then 16-byte stores to each destination.
 //
 // fp8: the same read, then per 128-column block amax (8 lanes, 16 columns
 // each, reduced with shuffles), scale = amax / 448 (IEEE division), each
