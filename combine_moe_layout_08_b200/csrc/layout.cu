@@ -175,36 +175,48 @@ struct RawIds {
 };
 
 // Fill the shared-memory cache of the tile's ids (16-byte loads when aligned),
-// zero the block's scratch and load the placement map.  Reads only the
+// zero the block's scratch and load the placement map.  With `order`, warp 0
+// loads the placement map and orders the experts by (partition, id) -- which
+// needs nothing else -- while the other warps do the rest.  Reads only the
 // caller's inputs.  Ends with a barrier.
-__device__ void stage_tile(const LayoutArgs& a, const Tile& tl, const Smem& S, RawIds& ids) {
-  const int tid = threadIdx.x;
+__device__ void stage_tile(const LayoutArgs& a, const Tile& tl, const Smem& S, RawIds& ids,
+                           bool order) {
   const int* src = a.idx + (size_t)tl.t0 * a.topk;
   ids.g = src;
   ids.s = nullptr;
-  if (tl.n_items <= a.key_cap) {
-    ids.s = S.keys;
-    const int n = tl.n_items;
-    if ((reinterpret_cast<uintptr_t>(src) & 15) == 0) {
-      const int n4 = n >> 2;
-      const int4* s4 = reinterpret_cast<const int4*>(src);
-      int4* k4 = reinterpret_cast<int4*>(S.keys);
+  const bool cache = tl.n_items <= a.key_cap;
+  if (cache) ids.s = S.keys;
+  if (order && warp_id() == 0) {
+    for (int e = lane_id(); e < a.G; e += kWarp) S.part_s[e] = __ldg(a.part_of + e);
+    __syncwarp();
+    expert_order_warp(S.part_s, a.G, a.E, S.pos, S.kcnt);
+  } else {
+    const int r = order ? (int)threadIdx.x - kWarp : (int)threadIdx.x;
+    const int nt = order ? kLThreads - kWarp : kLThreads;
+    if (cache) {
+      const int n = tl.n_items;
+      if ((reinterpret_cast<uintptr_t>(src) & 15) == 0) {
+        const int n4 = n >> 2;
+        const int4* s4 = reinterpret_cast<const int4*>(src);
+        int4* k4 = reinterpret_cast<int4*>(S.keys);
 #pragma unroll 4
-      for (int i = tid; i < n4; i += kLThreads) k4[i] = __ldg(s4 + i);
-      for (int i = (n4 << 2) + tid; i < n; i += kLThreads) S.keys[i] = __ldg(src + i);
-    } else {
+        for (int i = r; i < n4; i += nt) k4[i] = __ldg(s4 + i);
+        for (int i = (n4 << 2) + r; i < n; i += nt) S.keys[i] = __ldg(src + i);
+      } else {
 #pragma unroll 4
-      for (int i = tid; i < n; i += kLThreads) S.keys[i] = __ldg(src + i);
+        for (int i = r; i < n; i += nt) S.keys[i] = __ldg(src + i);
+      }
     }
+    if (!order)
+      for (int e = r; e < a.G; e += nt) S.part_s[e] = __ldg(a.part_of + e);
+    for (int i = r; i < kLWarps * a.G; i += nt) S.whist[i] = 0;
+    for (int i = r; i < a.W; i += nt) S.row[i] = 0;
+    for (int p = r; p < a.E; p += nt) {
+      S.pc[p] = 0;
+      S.pbase[p] = 0;
+    }
+    if (r < 4) S.misc[r] = 0;
   }
-  for (int e = tid; e < a.G; e += kLThreads) S.part_s[e] = __ldg(a.part_of + e);
-  for (int i = tid; i < kLWarps * a.G; i += kLThreads) S.whist[i] = 0;
-  for (int i = tid; i < a.W; i += kLThreads) S.row[i] = 0;
-  for (int p = tid; p < a.E; p += kLThreads) {
-    S.pc[p] = 0;
-    S.pbase[p] = 0;
-  }
-  if (tid < 4) S.misc[tid] = 0;
   __syncthreads();
 }
 
@@ -274,12 +286,6 @@ __device__ void rank_assign(int n, int K, int* whist, KeyOf key_of, OnRank on_ra
     __syncwarp();
   }
   __syncthreads();
-}
-
-// One warp: position of every expert in (partition, id) order, experts with
-// an invalid placement last.  Reads only the placement map.
-__device__ __forceinline__ void expert_order(const LayoutArgs& a, const Smem& S) {
-  expert_order_warp(S.part_s, a.G, a.E, S.pos, S.kcnt);
 }
 
 // Partition bit mask of token tl of the tile (valid pairs only).
@@ -471,9 +477,8 @@ __global__ void __launch_bounds__(kLThreads, kLMinBlocks) layout_cluster_kernel(
   pdl_wait();
   pdl_trigger();
   RawIds ids;
-  stage_tile(a, tl, S, ids);
+  stage_tile(a, tl, S, ids, true);
   count_tile(a, tl, S, ids, r == 0);
-  if (warp_id() == 0) expert_order(a, S);
   cluster.sync();
 
   // exchange: totals over the cluster and the prefix of the tiles before r
@@ -513,7 +518,7 @@ __global__ void __launch_bounds__(kLThreads, kLMinBlocks) layout_count_kernel(La
   pdl_wait();
   pdl_trigger();
   RawIds ids;
-  stage_tile(a, tl, S, ids);
+  stage_tile(a, tl, S, ids, false);
   count_tile(a, tl, S, ids, b == 0);
   int4* dst = reinterpret_cast<int4*>(a.tile_rows + (size_t)b * a.W);
   const int4* src = reinterpret_cast<const int4*>(S.row);
@@ -565,11 +570,11 @@ __global__ void __launch_bounds__(kLThreads, kLMinBlocks) layout_rank_kernel(Lay
   const Tile tl = tile_of(a, b);
   // Everything that depends only on the caller's inputs -- which were
   // complete before layout_count_kernel started -- runs before the wait:
-  // the tile's ids, its per-warp counts and the expert order.
+  // the tile's ids, the expert order (warp 0, meanwhile) and the tile's
+  // per-warp counts.
   RawIds ids;
-  stage_tile(a, tl, S, ids);
+  stage_tile(a, tl, S, ids, true);
   rank_count(tl.n_items, a.G, S.whist, nullptr, [&](int i) { return item_key(a, S, ids, i); });
-  if (warp_id() == 0) expert_order(a, S);
   pdl_wait();
   pdl_trigger();
 
