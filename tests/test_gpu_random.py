@@ -76,3 +76,50 @@ def test_random_problem(i):
         b.combine_two_level_(d["y"], g)
         torch.cuda.synchronize()
         assert compare_two_level(b, prob, d["y"], d["topk_weights"], d["topk_idx"], po, ref) == 0
+
+
+# duplicate expert ids inside a token (reading: separate rows, ranked by
+# slot), through the one-kernel and the separate schedules, the two-level
+# combine (duplicates fall in one partition group) and the tile metadata
+@pytest.mark.parametrize("M,topk,separate", [(200, 8, False), (200, 8, True), (3000, 4, False)])
+@pytest.mark.parametrize("pattern", ["one-expert", "few-experts", "one-partition"])
+def test_duplicate_expert_ids(M, topk, separate, pattern):
+    w = W.Workload("dups", M=M, N=256, G=16, topk=topk, E_part=8, routing="uniform",
+                   placement="contiguous", dedup=True, fp8=(topk == 4), seed=M + topk)
+    d = W.make_inputs(w, device=DEV)
+    rng = np.random.default_rng(M * 3 + topk)
+    po = W.make_placement(w)
+    if pattern == "one-expert":
+        idx = np.full((M, topk), 5, np.int32)
+    elif pattern == "few-experts":
+        idx = rng.integers(0, 3, size=(M, topk)).astype(np.int32)
+    else:
+        idx = rng.integers(0, 16, size=(M, topk)).astype(np.int32)
+        po = np.zeros_like(po)
+    prob = problem_of(w)
+    b = poisoned_buffers(prob, DEV)
+    b.tiles = moe.alloc_expert_tiles(prob, 16, DEV)
+    for t in (b.tiles.tile_first, b.tiles.tile_expert, b.tiles.tile_row, b.tiles.tile_rows):
+        t.fill_(POISON_I32)
+    idx_d, po_d, g = to_dev(idx), to_dev(po), to_dev(d["topk_weights"])
+    if separate:
+        b.layout_(idx_d, po_d)
+        b.dispatch_(d["x"])
+        b.expert_tiles_(po_d, 16)
+    else:
+        b.layout_dispatch_(idx_d, po_d, d["x"], block_m=16)
+    b.combine_(d["y"], g)
+    torch.cuda.synchronize()
+    ref = oracle.layout(idx, po, w.G, w.E_part, True)
+    compare_layout(b, ref, prob)
+    compare_dispatch_rows(b, prob, oracle.bf16_bits(d["x"]), ref["disp_token"])
+    untouched_rows_ok(b, ref["R_disp"])
+    assert compare_combine(b, prob, d["y"], d["topk_weights"], ref["exp_row"]) == 0
+    tiles = oracle.expert_tiles(ref["expert_count"], ref["expert_offset"], 16)
+    np.testing.assert_array_equal(b.tiles.tile_first.cpu().numpy(), tiles["tile_first"])
+    np.testing.assert_array_equal(b.tiles.tile_expert.cpu().numpy()[:tiles["n_tiles"]],
+                                  tiles["tile_expert"])
+    b.z = torch.empty((max(prob.capacity, 1), prob.N), dtype=torch.bfloat16, device=DEV)
+    b.combine_two_level_(d["y"], g)
+    torch.cuda.synchronize()
+    assert compare_two_level(b, prob, d["y"], d["topk_weights"], idx, po, ref) == 0
