@@ -172,13 +172,21 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # CPU oracle timing (the reference arm and the cpu_baseline leg)
 # ---------------------------------------------------------------------------
-def oracle_step_seconds(w, idx, po, gates, x_bits, y_bits):
+def oracle_step_seconds(w, idx, po, gates, x_bits, y_bits, stages=None):
+    """One oracle pass (layout, dispatch, combine); returns its seconds and
+    the layout, and adds each stage's seconds to ``stages`` if given."""
     import oracle
     t0 = time.perf_counter()
     lay = oracle.layout(idx, po, w.G, w.E_part, w.dedup)
+    t1 = time.perf_counter()
     oracle.dispatch(x_bits, lay["disp_token"], w.fp8)
+    t2 = time.perf_counter()
     oracle.combine(y_bits, gates, lay["exp_row"])
-    return time.perf_counter() - t0, lay
+    t3 = time.perf_counter()
+    if stages is not None:
+        for k, v in (("layout", t1 - t0), ("dispatch", t2 - t1), ("combine", t3 - t2)):
+            stages[k] = stages.get(k, 0.0) + v
+    return t3 - t0, lay
 
 
 def sample_workload(w: W.Workload, tokens: int):
@@ -573,18 +581,20 @@ def cpu_baseline(w, buf, idx_h, po_h, g_h, x, y, budget_s=10.0):
     ws = w.replace(M=m)
     xb = oracle.bf16_bits(x[:m])
     yb = oracle.bf16_bits(y[:m * w.topk])
-    times = []
+    times, stages = [], {}
     lay = None
     while sum(times) < budget_s and len(times) < 50:
-        t, lay = oracle_step_seconds(ws, idx_h[:m], po_h, g_h[:m], xb, yb)
+        t, lay = oracle_step_seconds(ws, idx_h[:m], po_h, g_h[:m], xb, yb, stages)
         times.append(t)
     b = sum(algorithmic_bytes(ws, lay["R_exp"], lay["R_disp"]).values())
     mean = sum(times) / len(times)
+    stage_ms = {k: round(v / len(times) * 1e3, 3) for k, v in stages.items()}
     what = f"full {w.name} problem (M={w.M})" if m == w.M else \
         f"first {m} of the {w.M} tokens of {w.name}"
     model, cores = host_cpu()
     return {"value": round(b / mean / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
             "tokens_per_s": round(m / mean, 1), "cpu": model, "host_cores": cores,
+            "ms_per_pass": stage_ms,
             "sample": f"{what}, {len(times)} oracle passes, {sum(times):.1f} s, single thread"}
 
 
