@@ -46,6 +46,9 @@ sys.path.insert(0, ROOT)
 import workloads as W  # noqa: E402
 
 DEFAULT_WORKLOAD = "M4096-zipf1.1"
+# batch sizes of the decode latency sweep: the M column of the latency table
+# of Triton-distributed issue #117 ("Results (Latency in us)")
+SWEEP_M = (2, 4, 8, 16, 32, 64, 128, 256, 512)
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
 
@@ -686,7 +689,7 @@ def run_latency_sweep(args):
     stream = torch.cuda.Stream(dev)
     flush_w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     rows = []
-    for M in (2, 4, 8, 16, 32, 64, 128, 256, 512):
+    for M in SWEEP_M:
         w = dataclasses.replace(base, name=f"decode-M{M}-uniform", M=M)
         d = W.make_inputs(w, device=dev)
         prob = moe.MoEProblem(w.M, w.N, w.G, w.topk, w.E_part, w.dedup, w.fp8)

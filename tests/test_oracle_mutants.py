@@ -18,6 +18,7 @@ from oracle import build as obuild
 
 import test_oracle_combine as C
 import test_oracle_fp8 as F
+import test_golden as GD
 import test_oracle_layout as L
 import test_oracle_tiles as T
 
@@ -94,6 +95,7 @@ def _pins():
         lambda: T.test_tiles_match_the_row_walk(1, 8, 2, 1, False, "random", 3),
         lambda: T.test_tiles_match_the_row_walk(200, 40, 8, 5, True, "random", 16),
         T.test_block_of_one_row_labels_every_row,
+        GD.test_zyphra_hot_pairs_closed_forms,
     ]
 
 
