@@ -198,3 +198,43 @@ def test_python_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(b, "build", lambda *a, **k: str(tmp_path / "absent.so"))
     with pytest.raises(RuntimeError):
         _lib.load()
+
+
+C_HOST = r"""
+#include <stdio.h>
+#include "moe_layout.h"
+
+int main(void) {
+    moe_problem_t p = {4096, 7168, 256, 8, 8, 0, 0};
+    moe_problem_t bad = {4096, 7, 256, 8, 8, 0, 0};
+    moe_layout_t lay = {0};
+    moe_tiles_t tiles = {0};
+    if (moe_abi_version() != MOE_ABI_VERSION) return 1;
+    if (moe_layout_workspace_size(&p) == 0 || moe_layout_workspace_size(&bad) != 0) return 2;
+    if (moe_expert_tiles_capacity(&p, 128) != (4096 * 8 + 127) / 128 + 256) return 3;
+    if (moe_layout_dispatch_fused(&p) != 0) return 4;
+    if (moe_status_string(MOE_ERR_ARG)[0] == 0) return 5;
+    /* invalid calls fail on the host, before any CUDA call */
+    if (moe_layout(&bad, 0, 0, &lay, 0, 0, 0) != MOE_ERR_ARG) return 6;
+    if (moe_expert_tiles(&p, 0, &lay, &tiles, 0) != MOE_ERR_ARG) return 7;
+    (void)moe_layout_static; (void)moe_dispatch; (void)moe_combine;
+    (void)moe_combine_partial; (void)moe_combine_reduce;
+    printf("ok\n");
+    return 0;
+}
+"""
+
+
+def test_plain_c_host_compiles_links_and_calls(tmp_path):
+    """The header is plain C99, and a C program links the library and calls
+    the entry points that need no GPU."""
+    libbuild.build()
+    src = tmp_path / "host.c"
+    exe = tmp_path / "host"
+    src.write_text(C_HOST)
+    lib_dir = os.path.dirname(_lib.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.dirname(HEADER), str(src),
+                    "-L", lib_dir, "-lmoe_layout", f"-Wl,-rpath,{lib_dir}", "-o", str(exe)],
+                   check=True, capture_output=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0 and out.stdout.strip() == "ok", (out.returncode, out.stderr)
