@@ -238,3 +238,18 @@ def test_plain_c_host_compiles_links_and_calls(tmp_path):
                    check=True, capture_output=True)
     out = subprocess.run([str(exe)], capture_output=True, text=True)
     assert out.returncode == 0 and out.stdout.strip() == "ok", (out.returncode, out.stderr)
+
+
+def test_header_compiles_as_cpp(tmp_path):
+    """The same host program as C++17: the header's extern "C" block keeps
+    the names unmangled, so it links against the library."""
+    libbuild.build()
+    src = tmp_path / "host.cpp"
+    exe = tmp_path / "host_cpp"
+    src.write_text(C_HOST)
+    lib_dir = os.path.dirname(_lib.LIB_PATH)
+    subprocess.run(["g++", "-std=c++17", "-Wall", "-Werror", "-I", os.path.dirname(HEADER),
+                    str(src), "-L", lib_dir, "-lmoe_layout", f"-Wl,-rpath,{lib_dir}", "-o", str(exe)],
+                   check=True, capture_output=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0 and out.stdout.strip() == "ok", (out.returncode, out.stderr)
