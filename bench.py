@@ -409,13 +409,16 @@ def run_ours(args, w):
         stream.synchronize()
         return [pev[i].elapsed_time(pev[i + 1]) for i in range(len(parts))]
 
-    for _ in range(max(args.warmup, 3)):
-        timed_step()
+    # NVTX ranges name the phases for a system-level profiler
+    nvtx = torch.cuda.nvtx.range
+    with nvtx("warm-up"):
+        for _ in range(max(args.warmup, 3)):
+            timed_step()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     step_ms = []
-    with ClockSampler(dev) as clk:
+    with ClockSampler(dev) as clk, nvtx("timed steps"):
         for _ in range(args.steps):
             step_ms.append(timed_step())
     torch.cuda.synchronize(dev)
@@ -424,14 +427,16 @@ def run_ours(args, w):
     total_ms = float(np.sum(step_ms))
     step_us = np.array(step_ms) * 1e3
     # per-kernel breakdown (untimed for the headline; same flush, same inputs)
-    for _ in range(3):
-        parts_step()
-    per = np.array([parts_step() for _ in range(args.steps)])   # [K, parts] ms
+    with nvtx("per-kernel breakdown"):
+        for _ in range(3):
+            parts_step()
+        per = np.array([parts_step() for _ in range(args.steps)])   # [K, parts] ms
     kern_ms = {name: float(per[:, i].mean()) for i, (name, _) in enumerate(parts)}
 
     # end to end through the public API with host buffers
-    e2e = run_e2e(args, wr, buf, idx_h, po_h, g_h, x, y, stream, dev, step_bytes,
-                  two_level, separate, bm)
+    with nvtx("end to end"):
+        e2e = run_e2e(args, wr, buf, idx_h, po_h, g_h, x, y, stream, dev, step_bytes,
+                      two_level, separate, bm)
 
     # aggregate over ranks: bytes and tokens summed, time = max
     (max_ms, max_e2e_ms), (all_bytes, all_tokens, all_e2e_bytes) = reduce_over_ranks(
