@@ -17,13 +17,19 @@ Each function follows a passage of the pages:
   accumulation);
 * :func:`combine_partial` / :func:`combine_reduce` -- the two-level combine
   of a deduplicated dispatch: per (token, partition) reduce in slot order,
-  then the token's sum over partitions in partition order.
+  then the token's sum over partitions in partition order;
+* :func:`expert_tiles` -- DeepSpeed PR #8180 "Key points": the per-tile
+  group map of a grouped GEMM over the expert rows, from the offsets.
 
-Pins (tests/test_oracle_*.py): pure-Python brute force of the layout
-definition on every tiny input, layout invariants, the e4m3 encoder against a
-nearest-value search of the format's decode table and against torch's
-float8_e4m3fn cast, bf16 rounding against torch, combine identities
-(one-hot / uniform weights) and a float64 bound.  Parity of the layout's
+Pins (tests/test_oracle_*.py, tests/test_golden.py): pure-Python brute force
+of the layout definition on every tiny input, layout invariants, the e4m3
+encoder against a nearest-value search of the format's decode table and
+against torch's float8_e4m3fn cast, bf16 rounding against torch, combine
+identities (one-hot / uniform weights) and float64 bounds for both combines,
+the tile metadata against a row walk over exp_row, and the dedup ratio of
+the hot-pairs batch against the closed form from the pages' statistics.
+Every pin set is checked to catch a list of plausible mistakes planted in a
+copy of the C source (tests/test_oracle_mutants.py).  Parity of the layout's
 row order, the dedup row order and the FP8 conventions (all-zero block,
 saturation) rests on stated readings of the pages, not on printed values.
 """
