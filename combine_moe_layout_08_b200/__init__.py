@@ -22,7 +22,7 @@ from typing import Optional
 import torch
 
 from . import _lib
-from ._lib import (MOE_MAX_E_PART, MOE_MAX_G, MOE_MAX_TOPK, MOE_STATIC_SCRATCH_BYTES,
+from ._lib import (MOE_MAX_E_PART, MOE_MAX_G, MOE_MAX_N, MOE_MAX_TOPK, MOE_STATIC_SCRATCH_BYTES,
                    MOE_STATUS_BAD_EXPERT,
                    MOE_STATUS_BAD_PART, MOE_STATUS_BAD_ROW, MoEError)
 
@@ -32,7 +32,7 @@ __all__ = ["MoEProblem", "MoELayout", "MoEBuffers", "MoEError", "alloc_layout",
            "expert_tiles_capacity", "alloc_expert_tiles", "ExpertTiles", "moe_combine", "moe_combine_partial", "moe_combine_reduce",
            "moe_status_string", "moe_abi_version", "MOE_STATUS_BAD_EXPERT",
            "MOE_STATUS_BAD_PART", "MOE_STATUS_BAD_ROW", "MOE_MAX_G", "MOE_MAX_E_PART",
-           "MOE_MAX_TOPK"]
+           "MOE_MAX_TOPK", "MOE_MAX_N"]
 
 
 @dataclasses.dataclass(frozen=True)

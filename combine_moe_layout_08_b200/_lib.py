@@ -18,6 +18,7 @@ MOE_ERR_ARG = 1
 MOE_ERR_WORKSPACE = 2
 MOE_ERR_CUDA = 3
 
+MOE_ABI_VERSION = 1
 MOE_STATUS_BAD_EXPERT = 1
 MOE_STATUS_BAD_PART = 2
 MOE_STATUS_BAD_ROW = 4
@@ -25,6 +26,7 @@ MOE_STATUS_BAD_ROW = 4
 MOE_MAX_G = 1024
 MOE_MAX_E_PART = 64
 MOE_MAX_TOPK = 32
+MOE_MAX_N = 1 << 24
 MOE_STATIC_SCRATCH_BYTES = 256 * 1024
 
 
@@ -102,6 +104,9 @@ def load():
             f = getattr(L, name)
             f.restype = res
             f.argtypes = args
+        if L.moe_abi_version() != MOE_ABI_VERSION:
+            raise RuntimeError(f"{LIB_PATH}: ABI version {L.moe_abi_version()}, the binding "
+                               f"expects {MOE_ABI_VERSION}; rebuild the library")
         _lib = L
         return L
 

@@ -13,7 +13,7 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 bool valid_problem(const moe_problem_t* p) {
   if (!p) return false;
-  if (p->M < 0 || p->N <= 0 || (p->N % 8) != 0) return false;
+  if (p->M < 0 || p->N <= 0 || p->N > MOE_MAX_N || (p->N % 8) != 0) return false;
   if (p->G < 1 || p->G > MOE_MAX_G) return false;
   if (p->topk < 1 || p->topk > MOE_MAX_TOPK) return false;
   if (p->E_part < 1 || p->E_part > MOE_MAX_E_PART) return false;

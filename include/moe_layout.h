@@ -58,13 +58,15 @@ typedef struct CUstream_st *moe_stream_t;
 #define MOE_MAX_G 1024
 #define MOE_MAX_E_PART 64
 #define MOE_MAX_TOPK 32
+#define MOE_MAX_N (1 << 24) /* columns: keeps every grid and in-row index in range */
 
 /*
  * Problem sizes, as the all-to-all benchmark of the Triton-distributed issue
  * #117 ("All2all performance comparison between Triton-distributed and
  * DeepEP", Benchmark Configuration) poses them:
  *   M       tokens (>= 0; M = 0 makes every call a no-op)
- *   N       hidden size, bf16 columns (> 0, multiple of 8; of 128 with fp8)
+ *   N       hidden size, bf16 columns (1..MOE_MAX_N, multiple of 8; of 128
+ *           with fp8)
  *   G       experts (1..MOE_MAX_G)
  *   topk    experts per token (1..MOE_MAX_TOPK); M*topk < 2^31
  *   E_part  destination partitions (1..MOE_MAX_E_PART)

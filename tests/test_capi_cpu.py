@@ -74,9 +74,11 @@ def test_workspace_size(L):
     W = (256 + 8 + 2 + 3) // 4 * 4
     assert big == ((nt * W * 4 + 255) // 256) * 256
     for bad in (P(N=7), P(G=0), P(G=1025), P(topk=0), P(topk=33), P(E_part=0), P(E_part=65),
-                P(M=-1), P(fp8=1, N=7176), P(dedup=2), P(M=1 << 28, topk=8)):
+                P(M=-1), P(fp8=1, N=7176), P(dedup=2), P(M=1 << 28, topk=8),
+                P(N=(1 << 24) + 8)):
         assert L.moe_layout_workspace_size(ctypes.byref(bad)) == 0
     assert L.moe_layout_workspace_size(None) == 0
+    assert L.moe_layout_workspace_size(ctypes.byref(P(N=1 << 24))) > 0   # the largest N
 
 
 no_gpu = pytest.mark.skipif(torch.cuda.is_available(), reason="fake pointers only without a GPU")
@@ -253,3 +255,11 @@ def test_header_compiles_as_cpp(tmp_path):
                    check=True, capture_output=True)
     out = subprocess.run([str(exe)], capture_output=True, text=True)
     assert out.returncode == 0 and out.stdout.strip() == "ok", (out.returncode, out.stderr)
+
+
+def test_python_constants_match_the_header():
+    src = open(HEADER).read()
+    defs = dict(re.findall(r"#define (MOE_\w+) \(?([^\s/]+)", src))
+    for name in ("MOE_MAX_G", "MOE_MAX_E_PART", "MOE_MAX_TOPK", "MOE_MAX_N", "MOE_STATUS_BAD_EXPERT",
+                 "MOE_STATUS_BAD_PART", "MOE_STATUS_BAD_ROW", "MOE_ABI_VERSION"):
+        assert eval(defs[name].rstrip(")")) == getattr(_lib, name), name
