@@ -259,7 +259,7 @@ def test_header_compiles_as_cpp(tmp_path):
 
 def test_python_constants_match_the_header():
     src = open(HEADER).read()
-    defs = dict(re.findall(r"#define (MOE_\w+) \(?([^\s/]+)", src))
+    defs = {k: v.strip() for k, v in re.findall(r"#define (MOE_\w+)[ \t]+([^/\n]+)", src)}
     for name in ("MOE_MAX_G", "MOE_MAX_E_PART", "MOE_MAX_TOPK", "MOE_MAX_N", "MOE_STATUS_BAD_EXPERT",
                  "MOE_STATUS_BAD_PART", "MOE_STATUS_BAD_ROW", "MOE_ABI_VERSION"):
-        assert eval(defs[name].rstrip(")")) == getattr(_lib, name), name
+        assert eval(defs[name]) == getattr(_lib, name), (name, defs[name])   # integer literals
