@@ -26,3 +26,15 @@ def test_every_traffic_record_names_existing_sources():
         assert r["bytes_per_launch"] > 0 and r["sources"]
         assert bench.source_digest(r["sources"])        # files exist and read
         assert os.path.exists(os.path.join(bench.ROOT, r["capture"])), r["capture"]
+
+
+def test_every_profile_summary_gives_its_command():
+    """Each ncu summary under profiles/ states the command that made it: an
+    ncu invocation of bench.py (a committed file) with --clock-control none."""
+    pdir = os.path.join(bench.ROOT, "profiles")
+    names = [n for n in os.listdir(pdir) if n.endswith(".md")]
+    assert names
+    for n in names:
+        text = open(os.path.join(pdir, n)).read()
+        assert "ncu " in text and "--clock-control none" in text, n
+        assert "python bench.py" in text, n
