@@ -7,8 +7,10 @@
 
 One step = one pass of the whole path over one batch: routing layout ->
 dispatch permute -> combine (libmoe_layout.so, through its C ABI), on the
-M = 4096, N = 7168, G = 256, topk = 8, E_part = 8, Zipf(1.1) workload by
-default.  Inputs are resident in HBM when the timed region starts.  Each
+largest workload by default: the prefill batch of M = 65536 tokens, N =
+7168, G = 256, topk = 8, E_part = 8, routing 50% uniform / 50% Zipf(1.2),
+per-partition dedup and the FP8 dispatch.  Inputs are resident in HBM when
+the timed region starts.  Each
 step is one CUDA-graph replay with events at its two ends on the device;
 a second graph of the same step with events between its parts gives the
 per-kernel breakdown.  L2 is flushed between steps (256 MiB written, then
@@ -45,7 +47,7 @@ sys.path.insert(0, ROOT)
 
 import workloads as W  # noqa: E402
 
-DEFAULT_WORKLOAD = "M4096-zipf1.1"
+DEFAULT_WORKLOAD = "prefill-M65536-mix-dedup-fp8"
 # batch sizes of the decode latency sweep: the M column of the latency table
 # of Triton-distributed issue #117 ("Results (Latency in us)")
 SWEEP_M = (2, 4, 8, 16, 32, 64, 128, 256, 512)
@@ -754,6 +756,9 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(W.WORKLOADS))
+    ap.add_argument("--tokens", type=int, default=0, metavar="M",
+                    help="run the workload's recipe at M tokens instead (a smaller case of the "
+                         "same kernels, e.g. for a profiler capture); named NAME@M<M>")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--schedule", choices=("auto", "separate"), default="auto",
                     help="separate: moe_layout + moe_dispatch even where one kernel does both")
@@ -769,6 +774,10 @@ def main(argv=None):
     if args.latency_sweep:
         return run_latency_sweep(args)
     w = W.get(args.workload)
+    if args.tokens:
+        if args.tokens < 1:
+            raise SystemExit("--tokens must be >= 1")
+        w = w.replace(name=f"{w.name}@M{args.tokens}", M=args.tokens)
     if args.impl == "reference":
         return run_reference(args, w)
     return run_ours(args, w)

@@ -158,8 +158,9 @@ def moe_layout_static(prob: MoEProblem, topk_idx: torch.Tensor, part_of: torch.T
     """moe_layout without a workspace argument, for callers that cannot
     allocate device memory: the scratch is a fixed device array inside the
     library (MOE_STATIC_SCRATCH_BYTES), shared by every call.  Calls that
-    overlap on the GPU race on it; the first call on a device must come
-    before any stream capture."""
+    overlap on the GPU race on it; the first call in each CUDA context (the
+    first on a device, and the first after its context was re-created) looks
+    up the array's address and must come before any stream capture."""
     dev = part_of.device
     _check(topk_idx, "topk_idx", torch.int32, prob.M * prob.topk, dev)
     _check(part_of, "part_of", torch.int32, prob.G, dev)

@@ -1,4 +1,5 @@
 // Host-side launch helpers shared by the kernels' translation units.
+#include <cuda.h>  // driver API types only: the two entry points below come through the runtime
 #include <cuda_runtime.h>
 
 #include <map>
@@ -8,6 +9,57 @@
 #include "moe_internal.h"
 
 namespace moe {
+
+namespace {
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+struct CtxFns {
+  CtxGetCurrentFn get_current = nullptr;
+  CtxGetIdFn get_id = nullptr;
+};
+
+// cuCtxGetCurrent and cuCtxGetId (CUDA 12.0), fetched once through the
+// runtime so that the library needs no link-time dependency on libcuda.
+const CtxFns& ctx_fns() {
+  static const CtxFns fns = [] {
+    CtxFns f;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      f.get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      f.get_id = reinterpret_cast<CtxGetIdFn>(p);
+    return f;
+  }();
+  return fns;
+}
+
+}  // namespace
+
+cudaError_t current_context_id(unsigned long long* id) {
+  const CtxFns& f = ctx_fns();
+  if (!f.get_current || !f.get_id) return cudaErrorNotSupported;
+  CUcontext ctx = nullptr;
+  if (f.get_current(&ctx) != CUDA_SUCCESS) return cudaErrorContextIsDestroyed;
+  if (!ctx) {
+    // No context is current on this thread yet: make the runtime's primary
+    // context of the current device current (cudaSetDevice initialises it).
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaSetDevice(dev);
+    if (e != cudaSuccess) return e;
+    if (f.get_current(&ctx) != CUDA_SUCCESS || !ctx) return cudaErrorDeviceUninitialized;
+  }
+  return f.get_id(ctx, id) == CUDA_SUCCESS ? cudaSuccess : cudaErrorContextIsDestroyed;
+}
 
 int device_block_slots(const void* kernel, int threads, size_t smem) {
   static std::mutex mu;
@@ -34,13 +86,16 @@ int device_block_slots(const void* kernel, int threads, size_t smem) {
 
 cudaError_t allow_dynamic_smem(const void* kernel, size_t bytes) {
   if (bytes <= 48 * 1024) return cudaSuccess;
-  static std::mutex mu;
-  static std::map<std::pair<int, const void*>, size_t> granted;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  // A kernel's attributes belong to the module loaded in one context: a
+  // context destroyed and re-created (cudaDeviceReset) starts from the
+  // defaults again, so what was granted is remembered per context.
+  unsigned long long ctx = 0;
+  cudaError_t e = current_context_id(&ctx);
   if (e != cudaSuccess) return e;
+  static std::mutex mu;
+  static std::map<std::pair<unsigned long long, const void*>, size_t> granted;
   std::lock_guard<std::mutex> lock(mu);
-  size_t& g = granted[std::make_pair(dev, kernel)];
+  size_t& g = granted[std::make_pair(ctx, kernel)];
   if (g >= bytes) return cudaSuccess;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
   if (e == cudaSuccess) g = bytes;

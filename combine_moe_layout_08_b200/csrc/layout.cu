@@ -596,15 +596,18 @@ size_t smem_bytes(const moe_problem_t& p, int key_cap) {
 
 }  // namespace
 
+// In 64 bits: M may be as large as 2^31 - 1 (topk = E_part = 1), where
+// M + 147 no longer fits an int.  The results do (T <= 2^31 / 148 + 32,
+// at most 148 tiles).
 int layout_tile_tokens(int M) {
-  int t = (M + 147) / 148;
+  int64_t t = ((int64_t)M + 147) / 148;
   t = (t + 31) / 32 * 32;
-  return std::max(MOE_TILE_MIN_TOKENS, t);
+  return (int)std::max<int64_t>(MOE_TILE_MIN_TOKENS, t);
 }
 
 int layout_num_tiles(int M) {
-  const int T = layout_tile_tokens(M);
-  return std::max(1, (M + T - 1) / T);
+  const int64_t T = layout_tile_tokens(M);
+  return (int)std::max<int64_t>(1, ((int64_t)M + T - 1) / T);
 }
 
 size_t layout_workspace_bytes(const moe_problem_t& p) {

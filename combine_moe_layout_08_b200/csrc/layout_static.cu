@@ -9,10 +9,14 @@
 // array (kMoeStaticScratchBytes) until the process exits.
 //
 // The array's name in host code is only a host-side stand-in, not a device
-// address, so the device address is looked up with cudaGetSymbolAddress once
-// per device (with that device current) on the first call made on it, and
-// then passed to the kernels like any other workspace.  The first call on a
-// device therefore does this set-up and should come before any stream
+// address, so the device address is looked up with cudaGetSymbolAddress, with
+// the device current, and then passed to the kernels like any other
+// workspace.  The address belongs to the module loaded in one CUDA context:
+// it is looked up on the first call in each context (the process's first
+// call on a device, and the first call after that device's context was
+// destroyed and re-created, e.g. by cudaDeviceReset) and remembered under the
+// context's id, which is never reused within a process, so a stale address is
+// never handed to a kernel.  Such a first call should come before any stream
 // capture.
 //
 // All calls share the one array and it keeps the last call's contents.  The
@@ -23,6 +27,7 @@
 #include <cuda_runtime.h>
 
 #include <mutex>
+#include <unordered_map>
 
 #include "moe_internal.h"
 #include "moe_layout.h"
@@ -30,27 +35,26 @@
 namespace {
 
 constexpr size_t kMoeStaticScratchBytes = MOE_STATIC_SCRATCH_BYTES;
-constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_layout_scratch[kMoeStaticScratchBytes];
 
 std::mutex g_setup_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
+std::unordered_map<unsigned long long, void*> g_scratch_addr;  // context id -> address
 
-// Device address of g_layout_scratch on the current device (looked up once).
+// Device address of g_layout_scratch in the current context.
 cudaError_t scratch_address(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  unsigned long long ctx = 0;
+  cudaError_t e = moe::current_context_id(&ctx);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (!g_scratch_addr[dev]) {
+  auto it = g_scratch_addr.find(ctx);
+  if (it == g_scratch_addr.end()) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_layout_scratch);
     if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = p;
+    it = g_scratch_addr.emplace(ctx, p).first;
   }
-  *out = g_scratch_addr[dev];
+  *out = it->second;
   return cudaSuccess;
 }
 

@@ -45,8 +45,13 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-// Raise `kernel`'s dynamic shared-memory limit on the current device to at
-// least `bytes` (once per device and kernel; no-op up to 48 KB).
+// Unique id of the CUDA context current on this thread (cuCtxGetId; ids are
+// never reused within a process, so a context destroyed and re-created gets
+// a new one).  Makes the current device's primary context current if none is.
+cudaError_t current_context_id(unsigned long long* id);
+
+// Raise `kernel`'s dynamic shared-memory limit in the current context to at
+// least `bytes` (once per context and kernel; no-op up to 48 KB).
 cudaError_t allow_dynamic_smem(const void* kernel, size_t bytes);
 
 // Tokens per layout tile: about one tile per SM, at least

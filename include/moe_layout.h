@@ -167,14 +167,18 @@ int moe_layout(const moe_problem_t *prob, const int32_t *topk_idx,
  *   library, held by every GPU that loads it until the process exits.
  *   Limit: a problem whose moe_layout_workspace_size() exceeds
  *   MOE_STATIC_SCRATCH_BYTES is rejected with MOE_ERR_WORKSPACE before any
- *   launch.  The layout uses at most 148 tiles of G + E_part + 2 ints each
- *   (padded to 4), so every M fits when G + E_part <= 438 (G = 256,
- *   E_part = 8 always fits); larger G fit only for small M.
- *   The first call on a device looks up the array's device address (one
- *   cudaGetSymbolAddress with that device current); make it before any
- *   stream capture.  Every call shares the array: calls whose execution
- *   overlaps on the GPU (other streams, other threads) race -- serialise them.
- *   Nothing in the array needs to start at zero.
+ *   launch.  The layout uses at most 148 tiles of G + 2 ints each, plus
+ *   E_part more with dedup (padded to 4), so every M fits when
+ *   G + (dedup ? E_part : 0) <= 438 (G = 256, E_part = 8 always fits);
+ *   larger G fit only for small M.
+ *   The first call in each CUDA context looks up the array's device address
+ *   (one cudaGetSymbolAddress with the device current): the process's first
+ *   call on a device, and the first call after that device's context was
+ *   destroyed and re-created (cudaDeviceReset).  The address is remembered
+ *   per context, never reused for another one.  Make such a first call
+ *   before any stream capture.  Every call shares the array: calls whose
+ *   execution overlaps on the GPU (other streams, other threads) race --
+ *   serialise them.  Nothing in the array needs to start at zero.
  *   Other arguments, errors and results as moe_layout.
  */
 #define MOE_STATIC_SCRATCH_BYTES (256 * 1024)

@@ -157,3 +157,130 @@ def compare_two_level(b: moe.MoEBuffers, prob, y_dev, gates, idx, part_of, ref, 
     d = ulp_distance_bf16(got, out_ref)
     assert d.max(initial=0) <= max_ulp, f"two-level combine differs by {d.max()} bf16 steps"
     return int(np.count_nonzero(got != out_ref))
+
+
+# ---------------------------------------------------------------------------
+# element-by-element comparison of a large batch, in chunks
+# ---------------------------------------------------------------------------
+def run_chunks(jobs, workers=None, in_flight=None):
+    """``jobs`` yields (label, check, args): the device -> host gathers run
+    in the caller's thread as the generator advances, each ``check(*args)``
+    (oracle + comparison, plain C through ctypes, which releases the GIL) in
+    a pool of threads.  At most ``in_flight`` gathered chunks are held at
+    once.  Returns the results in order; the first failing check raises."""
+    import os
+    import threading
+    from concurrent.futures import ThreadPoolExecutor
+    workers = workers or max(1, min(32, len(os.sched_getaffinity(0))))
+    gate = threading.BoundedSemaphore(in_flight or workers + 2)
+    futs = []
+
+    def wrapped(label, check, args):
+        try:
+            return check(*args)
+        except AssertionError as e:
+            raise AssertionError(f"{label}: {e}") from None
+        finally:
+            gate.release()
+
+    with ThreadPoolExecutor(workers) as ex:
+        for label, check, args in jobs:
+            gate.acquire()
+            futs.append(ex.submit(wrapped, label, check, args))
+        return [f.result() for f in futs]
+
+
+def _check_dispatch_chunk(x_bits, dt, fp8, got, got_scale):
+    if fp8:
+        q, s = oracle.dispatch(x_bits, dt, True)
+        np.testing.assert_array_equal(got, q)
+        np.testing.assert_array_equal(got_scale.view(np.uint32), s.view(np.uint32))
+    else:
+        np.testing.assert_array_equal(got, oracle.dispatch(x_bits, dt, False))
+    return dt.shape[0]
+
+
+def dispatch_all_rows(b: moe.MoEBuffers, prob, x_bits, disp_token, rows_per_chunk=8192):
+    """Every dispatch row [0, R_disp) (bytes, and scales with FP8) bit-exact
+    against the oracle; returns the number of rows compared."""
+    R = disp_token.shape[0]
+
+    def jobs():
+        for r0 in range(0, R, rows_per_chunk):
+            r1 = min(R, r0 + rows_per_chunk)
+            got = b.recv_x[r0:r1]
+            got = got.cpu().numpy() if prob.fp8 else \
+                got.view(torch.int16).cpu().numpy().view(np.uint16)
+            gs = b.recv_scale[r0:r1].cpu().numpy() if prob.fp8 else None
+            yield f"dispatch rows [{r0}, {r1})", _check_dispatch_chunk, \
+                (x_bits, disp_token[r0:r1], prob.fp8, got, gs)
+
+    return sum(run_chunks(jobs()))
+
+
+def _check_combine_chunk(y_sub, gates, er_sub, got, max_ulp):
+    want = oracle.combine(y_sub, gates, er_sub)
+    d = ulp_distance_bf16(got, want)
+    assert d.max(initial=0) <= max_ulp, f"combine differs by {d.max()} bf16 steps"
+    return int(np.count_nonzero(got != want))
+
+
+def _gather_rows(t: torch.Tensor, rows: np.ndarray) -> np.ndarray:
+    return oracle.bf16_bits(t[torch.from_numpy(rows.astype(np.int64)).to(t.device)])
+
+
+def combine_all_tokens(b: moe.MoEBuffers, y_dev, gates, exp_row, tokens_per_chunk=1024, max_ulp=1):
+    """Every out row within max_ulp bf16 steps of the oracle; returns the
+    number of elements that differ at all (expected 0)."""
+    M, topk = exp_row.shape
+
+    def jobs():
+        for t0 in range(0, M, tokens_per_chunk):
+            t1 = min(M, t0 + tokens_per_chunk)
+            er = exp_row[t0:t1]
+            valid = er >= 0
+            y_sub = _gather_rows(y_dev, np.where(valid, er, 0).ravel())
+            er_sub = np.where(valid, np.arange(er.size).reshape(er.shape), -1).astype(np.int32)
+            got = oracle.bf16_bits(b.out[t0:t1])
+            yield f"combine tokens [{t0}, {t1})", _check_combine_chunk, \
+                (y_sub, gates[t0:t1], er_sub, got, max_ulp)
+
+    return sum(run_chunks(jobs()))
+
+
+def _check_two_level_chunk(y_sub, gates, idx, part_of, er_sub, dr_sub, z_got, z_sel, got, max_ulp):
+    n, E = dr_sub.shape
+    lay_sub = dict(exp_row=er_sub, disp_row=dr_sub, R_disp=n * E)
+    z_ref = oracle.combine_partial(y_sub, gates, idx, part_of, lay_sub)
+    out_ref = oracle.combine_reduce(z_ref, dr_sub)
+    np.testing.assert_array_equal(z_got, z_ref[z_sel])
+    d = ulp_distance_bf16(got, out_ref)
+    assert d.max(initial=0) <= max_ulp, f"two-level combine differs by {d.max()} bf16 steps"
+    return int(np.count_nonzero(got != out_ref))
+
+
+def two_level_all_tokens(b: moe.MoEBuffers, prob, y_dev, gates, idx, part_of, ref,
+                         tokens_per_chunk=1024, max_ulp=1):
+    """Two-level combine of every token: all z rows bit-exact, every out row
+    within max_ulp bf16 steps; returns the out elements that differ."""
+    M, topk = idx.shape
+    E = prob.E_part
+
+    def jobs():
+        for t0 in range(0, M, tokens_per_chunk):
+            t1 = min(M, t0 + tokens_per_chunk)
+            n = t1 - t0
+            er = ref["exp_row"][t0:t1]
+            dr = ref["disp_row"][t0:t1]
+            valid = er >= 0
+            y_sub = _gather_rows(y_dev, np.where(valid, er, 0).ravel())
+            er_sub = np.where(valid, np.arange(n * topk).reshape(n, topk), -1).astype(np.int32)
+            dvalid = dr >= 0
+            dr_sub = np.where(dvalid, np.arange(n * E).reshape(n, E), -1).astype(np.int32)
+            z_got = _gather_rows(b.z, dr[dvalid])
+            got = oracle.bf16_bits(b.out[t0:t1])
+            yield f"two-level tokens [{t0}, {t1})", _check_two_level_chunk, \
+                (y_sub, gates[t0:t1], idx[t0:t1], part_of, er_sub, dr_sub, z_got, dr_sub[dvalid],
+                 got, max_ulp)
+
+    return sum(run_chunks(jobs()))

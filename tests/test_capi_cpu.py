@@ -81,6 +81,38 @@ def test_workspace_size(L):
     assert L.moe_layout_workspace_size(ctypes.byref(P(N=1 << 24))) > 0   # the largest N
 
 
+def _expected_workspace(M, G, E, dedup):
+    """One row per tile of T tokens, T = max(128, ceil(M / 148) rounded up to
+    32), rows of G (+ E with dedup) + 2 ints padded to 4, rounded to 256 B;
+    Python integers, so nothing overflows."""
+    T = max(128, -(-(-(-M // 148)) // 32) * 32)
+    nt = max(1, -(-M // T))
+    W = -(-(G + (E if dedup else 0) + 2) // 4) * 4
+    return -(-(nt * W * 4) // 256) * 256, nt
+
+
+@pytest.mark.parametrize("topk,E,dedup", [(1, 1, 0), (1, 1, 1), (2, 1, 0), (1, 2, 1)])
+def test_workspace_size_at_the_largest_batch(L, topk, E, dedup):
+    """M up to the admitted limit (M*topk and M*E_part below 2^31): the tile
+    arithmetic must not overflow 32 bits, and one past the limit is refused."""
+    top = (1 << 31) - 1
+    M = min(top // topk, top // E)
+    for G in (1, 256, 1024):
+        want, nt = _expected_workspace(M, G, E, dedup)
+        assert nt == 148
+        got = L.moe_layout_workspace_size(ctypes.byref(P(M=M, N=8, G=G, topk=topk, E_part=E,
+                                                         dedup=dedup)))
+        assert got == want, (M, G, got, want)
+    assert L.moe_layout_workspace_size(ctypes.byref(P(M=M + 1, N=8, G=8, topk=topk, E_part=E,
+                                                      dedup=dedup))) == 0
+    # every M just below the limit, including those where M + 147 passes 2^31
+    for m in (M - 1, M - 100, M - 147, M - 148, M - 200, min(M, (1 << 31) - 148 * 32)):
+        want, _ = _expected_workspace(m, 64, E, dedup)
+        got = L.moe_layout_workspace_size(ctypes.byref(P(M=m, N=8, G=64, topk=topk, E_part=E,
+                                                         dedup=dedup)))
+        assert got == want, (m, got, want)
+
+
 no_gpu = pytest.mark.skipif(torch.cuda.is_available(), reason="fake pointers only without a GPU")
 
 FAKE = 0x7f0000000000  # never dereferenced: every call below fails validation
