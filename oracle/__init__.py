@@ -19,7 +19,11 @@ Each function follows a passage of the pages:
   of a deduplicated dispatch: per (token, partition) reduce in slot order,
   then the token's sum over partitions in partition order;
 * :func:`expert_tiles` -- DeepSpeed PR #8180 "Key points": the per-tile
-  group map of a grouped GEMM over the expert rows, from the offsets.
+  group map of a grouped GEMM over the expert rows, from the offsets;
+* :func:`ep_plan` -- the counts exchange of an expert-parallel all-to-all
+  (issue #117 test snippet: split_send_buf -> split_recv_buf,
+  send_split_cumsum) into Purlin's transposed-V receive layout (section 3.1:
+  destination r holds partition r of every source, in source-rank order).
 
 Pins (tests/test_oracle_*.py, tests/test_golden.py): pure-Python brute force
 of the layout definition on every tiny input, layout invariants, the e4m3
@@ -73,6 +77,8 @@ def lib():
         L.oracle_combine_partial.argtypes = [ctypes.c_int32] * 4 + [ctypes.c_int64] + [ctypes.c_void_p] * 8
         L.oracle_expert_tiles.restype = ctypes.c_int64
         L.oracle_expert_tiles.argtypes = [ctypes.c_int32, ctypes.c_int32] + [ctypes.c_void_p] * 6
+        L.oracle_ep_plan.restype = None
+        L.oracle_ep_plan.argtypes = [ctypes.c_int32] * 3 + [ctypes.c_void_p] * 10
         L.oracle_combine_reduce.restype = ctypes.c_int
         L.oracle_combine_reduce.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int64] + [ctypes.c_void_p] * 4
         _lib = L
@@ -233,6 +239,40 @@ def expert_tiles(expert_count, expert_offset, block_m: int) -> dict:
     return dict(tile_first=first, tile_expert=te[:n], tile_row=tr[:n], tile_rows=tn[:n], n_tiles=n)
 
 
+def ep_plan(part_counts, rank: int, expert_counts=None, part_of=None) -> dict:
+    """Exchange plan of ``rank`` among W ranks from every rank's per-partition
+    row counts ``part_counts`` [W, W] (row s: rank s's part_count) and,
+    optionally, every rank's expert counts ``expert_counts`` [W, G] with the
+    placement ``part_of`` [G] (expert -> rank).  Returns int32 arrays
+    send_offset [W], src_offset [W], recv_count [W], recv_offset [W+1], and
+    with expert counts recv_expert_count [G] and recv_block_offset [W, G];
+    plus the status word (8: counts negative, too large or inconsistent)."""
+    P = _c(part_counts, np.int32)
+    W = P.shape[0]
+    assert P.shape == (W, W) and 0 <= rank < W
+    out = dict(send_offset=np.zeros(W, np.int32), src_offset=np.zeros(W, np.int32),
+               recv_count=np.zeros(W, np.int32), recv_offset=np.zeros(W + 1, np.int32))
+    X = po = rec = blk = None
+    G = 0
+    if expert_counts is not None:
+        X = _c(expert_counts, np.int32)
+        G = X.shape[1]
+        assert X.shape == (W, G)
+        po = _c(part_of, np.int32)
+        assert po.shape == (G,)
+        rec = np.zeros(G, np.int32)
+        blk = np.zeros((W, G), np.int32)
+    st = np.zeros(1, np.int32)
+    lib().oracle_ep_plan(W, rank, G, _p(P), _p(X), _p(po), _p(out["send_offset"]),
+                         _p(out["src_offset"]), _p(out["recv_count"]), _p(out["recv_offset"]),
+                         _p(rec), _p(blk), _p(st))
+    if X is not None:
+        out["recv_expert_count"] = rec
+        out["recv_block_offset"] = blk
+    out["status"] = int(st[0])
+    return out
+
+
 def bf16_round(values) -> np.ndarray:
     """float32 -> bf16 bits (uint16), nearest-even."""
     v = _c(values, np.float32).ravel()
@@ -269,7 +309,7 @@ def bits_to_f32(b) -> np.ndarray:
 
 
 __all__ = ["layout", "dispatch", "combine", "combine_partial", "combine_reduce",
-           "bf16_round", "e4m3_encode", "step",
+           "expert_tiles", "ep_plan", "bf16_round", "e4m3_encode", "step",
            "bf16_bits", "bits_to_f32", "STATUS_BAD_EXPERT", "STATUS_BAD_PART",
            "lib"]
 

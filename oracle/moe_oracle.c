@@ -32,6 +32,16 @@
  *                w[t,k] * y[exp_row[t,k], c]) in fp32 starting from +0.
  *   tiles     -- DeepSpeed PR #8180, "Key points": the per-tile -> group map
  *                of a grouped GEMM over the expert rows, from the offsets.
+ *   ep_plan   -- the counts exchange of an expert-parallel all-to-all over W
+ *                ranks (partition p = rank p): Triton-distributed issue #117,
+ *                test snippet (split_send_buf -> split_recv_buf,
+ *                send_split_cumsum), and Purlin section 3.1, the transposed-V
+ *                layout: destination r receives partition r of every source
+ *                and arranges it in source-rank order.  From the matrix of
+ *                every rank's per-partition row counts it gives each rank's
+ *                offsets: where its rows go in every destination, where its
+ *                rows start in every source, where every source's rows land
+ *                in its own receive buffer, and per (source, expert) blocks.
  *
  * Invalid input (expert id outside [0, G), placement entry outside
  * [0, E_part)) is never an error of the call: the offending pairs are left out
@@ -475,4 +485,95 @@ int64_t oracle_expert_tiles(int32_t G, int32_t block_m, const int32_t *expert_co
         }
     }
     return total;
+}
+
+/* ------------------------------------------------------------------------ */
+/* expert-parallel exchange plan (counts exchange)                          */
+/* ------------------------------------------------------------------------ */
+
+#define ORACLE_BAD_COUNT 8
+
+/* Stores v, or -1 and the status bit if v is negative or does not fit an int32. */
+static int32_t orc_fit(int64_t v, int32_t *status)
+{
+    if (v < 0 || v > INT32_MAX) {
+        *status |= ORACLE_BAD_COUNT;
+        return -1;
+    }
+    return (int32_t)v;
+}
+
+/*
+ * Plan of rank r of W for the exchange of dispatch rows.
+ *   part_counts   [W][W]: row s = part_count of rank s's layout (rows that s
+ *                 sends to each destination d)
+ *   expert_counts [W][G] or NULL: row s = expert_count of rank s's layout
+ *                 (without dedup, where dispatch rows are expert rows)
+ *   part_of       [G]: rank of each expert (used with expert_counts)
+ * Outputs, each a plain sum written out:
+ *   send_offset[d]  = sum_{s<r} part_counts[s][d]   (r's rows start here in d's buffer)
+ *   src_offset[s]   = sum_{d<r} part_counts[s][d]   (rows for r start here in s's buffer)
+ *   recv_count[s]   = part_counts[s][r]
+ *   recv_offset[s]  = sum_{s'<s} part_counts[s'][r], recv_offset[W] = sum over all s
+ * and with expert_counts, for every expert e:
+ *   recv_expert_count[e]    = sum_s expert_counts[s][e] if part_of[e] == r, else 0
+ *   recv_block_offset[s][e] = recv_offset[s] + sum of expert_counts[s][f] over the
+ *                             experts f < e with part_of[f] == r, if part_of[e] == r,
+ *                             else -1
+ *   (a source's rows for r are its expert rows of partition r, in expert-id order)
+ * Negative counts, sums past INT32_MAX and, with expert_counts, a source whose
+ * expert counts on r do not add up to part_counts[s][r] set bit 8 of *status.
+ */
+void oracle_ep_plan(int32_t W, int32_t r, int32_t G, const int32_t *part_counts,
+                    const int32_t *expert_counts, const int32_t *part_of,
+                    int32_t *send_offset, int32_t *src_offset, int32_t *recv_count,
+                    int32_t *recv_offset, int32_t *recv_expert_count,
+                    int32_t *recv_block_offset, int32_t *status)
+{
+    int32_t st = 0;
+    for (int64_t i = 0; i < (int64_t)W * W; ++i)
+        if (part_counts[i] < 0) st |= ORACLE_BAD_COUNT;
+    for (int32_t d = 0; d < W; ++d) {
+        int64_t sum = 0;
+        for (int32_t s = 0; s < r; ++s) sum += part_counts[(int64_t)s * W + d];
+        send_offset[d] = orc_fit(sum, &st);
+    }
+    for (int32_t s = 0; s < W; ++s) {
+        int64_t sum = 0;
+        for (int32_t d = 0; d < r; ++d) sum += part_counts[(int64_t)s * W + d];
+        src_offset[s] = orc_fit(sum, &st);
+        recv_count[s] = part_counts[(int64_t)s * W + r];
+    }
+    for (int32_t s = 0; s <= W; ++s) {
+        int64_t sum = 0;
+        for (int32_t q = 0; q < s; ++q) sum += part_counts[(int64_t)q * W + r];
+        recv_offset[s] = orc_fit(sum, &st);
+    }
+    if (expert_counts) {
+        for (int32_t e = 0; e < G; ++e) {
+            int64_t sum = 0;
+            if (part_of[e] == r)
+                for (int32_t s = 0; s < W; ++s) sum += expert_counts[(int64_t)s * G + e];
+            recv_expert_count[e] = orc_fit(sum, &st);
+        }
+        for (int32_t s = 0; s < W; ++s) {
+            int64_t on_r = 0;
+            for (int32_t e = 0; e < G; ++e) {
+                const int64_t c = expert_counts[(int64_t)s * G + e];
+                if (c < 0) st |= ORACLE_BAD_COUNT;
+                if (part_of[e] != r) {
+                    recv_block_offset[(int64_t)s * G + e] = -1;
+                    continue;
+                }
+                int64_t before = 0;
+                for (int32_t f = 0; f < e; ++f)
+                    if (part_of[f] == r) before += expert_counts[(int64_t)s * G + f];
+                recv_block_offset[(int64_t)s * G + e] =
+                    orc_fit((int64_t)recv_offset[s] + before, &st);
+                on_r += c;
+            }
+            if (on_r != part_counts[(int64_t)s * W + r]) st |= ORACLE_BAD_COUNT;
+        }
+    }
+    *status = st;
 }

@@ -17,6 +17,7 @@ import oracle
 from oracle import build as obuild
 
 import test_oracle_combine as C
+import test_oracle_ep as EP
 import test_oracle_fp8 as F
 import test_golden as GD
 import test_oracle_layout as L
@@ -64,6 +65,18 @@ MUTANTS = [
     ("tiles: full last tile", "int64_t oracle_expert_tiles", "(rest < block_m ? rest : block_m)", "(block_m)"),
     ("tiles: row start", "int64_t oracle_expert_tiles", "(expert_offset[e] + j * block_m)",
      "(expert_offset[e] + j * block_m + (j > 0))"),
+    ("ep: send offset counts own rank", "void oracle_ep_plan", "for (int32_t s = 0; s < r; ++s)",
+     "for (int32_t s = 0; s <= r; ++s)"),
+    ("ep: source offset transposed", "void oracle_ep_plan",
+     "for (int32_t d = 0; d < r; ++d) sum += part_counts[(int64_t)s * W + d];",
+     "for (int32_t d = 0; d < r; ++d) sum += part_counts[(int64_t)d * W + s];"),
+    ("ep: receive offsets transposed", "void oracle_ep_plan",
+     "for (int32_t q = 0; q < s; ++q) sum += part_counts[(int64_t)q * W + r];",
+     "for (int32_t q = 0; q < s; ++q) sum += part_counts[(int64_t)r * W + q];"),
+    ("ep: receive count row", "void oracle_ep_plan", "recv_count[s] = part_counts[(int64_t)s * W + r];",
+     "recv_count[s] = part_counts[(int64_t)r * W + s];"),
+    ("ep: block counts its own expert", "void oracle_ep_plan", "for (int32_t f = 0; f < e; ++f)",
+     "for (int32_t f = 0; f <= e; ++f)"),
 ]
 
 
@@ -96,6 +109,10 @@ def _pins():
         lambda: T.test_tiles_match_the_row_walk(200, 40, 8, 5, True, "random", 16),
         T.test_block_of_one_row_labels_every_row,
         GD.test_zyphra_hot_pairs_closed_forms,
+        lambda: EP.test_exchange_by_definition_push_and_pull(3, 2, 12, 2, False),
+        lambda: EP.test_exchange_by_definition_push_and_pull(4, 3, 16, 4, True),
+        lambda: EP.test_expert_blocks_hold_each_sources_expert_rows(4, 3, 16, 4),
+        EP.test_closed_forms,
     ]
 
 
