@@ -20,6 +20,11 @@ namespace moe {
 namespace {
 
 constexpr int kCThreads = 128;
+// Compile-time tuning constant: topk 5..8 batches of at most this many routed
+// pairs gather all their slots in one round (0: never).
+#ifndef MOE_COMBINE_ONE_ROUND_ITEMS
+#define MOE_COMBINE_ONE_ROUND_ITEMS 0
+#endif
 
 struct CombineArgs {
   const uint4* __restrict__ y;  // [cap][N8]
@@ -47,6 +52,14 @@ __global__ void __launch_bounds__(kCThreads) combine_kernel(CombineArgs a) {
   __shared__ float wts[MOE_MAX_TOPK];
   const int t = blockIdx.x;
   const int tid = threadIdx.x;
+  // The gates are the router's output, not the previous kernel's: warm L2
+  // with the token's row while that kernel may still run (a prefetch is
+  // safe before the wait, see prefetch_line_l2).
+  if (tid == 0) {
+    const float* g = a.w + (size_t)t * a.topk;
+    prefetch_line_l2(g);
+    prefetch_line_l2(g + a.topk - 1);
+  }
   pdl_wait();
   pdl_trigger();
   if (tid < a.topk) {
@@ -128,6 +141,10 @@ cudaError_t launch_combine(const moe_problem_t& p, const void* y, const float* w
   // (combine us at topk 8, M4096 / M8192 / M65536): KG = 4 beats 8, 2 and 1
   // (90.2 / 170.3 / 1290 against 90.6 / 172.5 / 1307 for 8, 91.3 / 174.0 /
   // 1316 for 2); at topk 2, U = 4 beats 2 and 1.
+  // Small batches are bound by latency, not bandwidth: all slots (up to 8)
+  // in one round trip to memory instead of two.
+  if (p.topk >= 5 && p.topk <= 8 && (int64_t)p.M * p.topk <= MOE_COMBINE_ONE_ROUND_ITEMS)
+    return launch<8, 1>(a, p.M, stream);
   if (p.topk >= 5) return launch<4, 1>(a, p.M, stream);
   if (p.topk >= 3) return launch<4, 2>(a, p.M, stream);
   if (p.topk == 2) return launch<2, 4>(a, p.M, stream);

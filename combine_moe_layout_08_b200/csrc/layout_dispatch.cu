@@ -2,35 +2,50 @@
 // kernel.  At a few hundred tokens the tiled layout and the dispatch are
 // bound by latency, not bandwidth (Triton-distributed issue #117, "Results
 // (Latency in us)": M = 2..512 at N = 7168, G = 256, topk = 8), so this
-// schedule removes a launch and every inter-block step: each block recomputes
-// the whole (small) layout in shared memory from all routing ids, derives the
-// rows of its own chunk of T consecutive tokens and copies their rows there.
-// No block waits for another.  T = ceil(M / 148) keeps the grid at about one
-// block per SM.
+// schedule has no inter-block step at all and as few block-wide phases as
+// the layout allows.
 //
-// Block (b, y) of 512 threads, chunk tokens [t0, t0 + nt), t0 = b * T:
-//   1. issues the loads of its slice of x[t0 .. t0 + nt) -- the chunk's rows
-//      are contiguous, so thread i holds flat vectors i, i + 512, ... --
-//      while the layout is computed;
+// Every index of the layout is a rank.  Give each routed pair i = t * topk + k
+// whose expert e is valid (e in [0, G), placed on a partition p in
+// [0, E_part)) the sort key  K_i = (p * G + e) << 13 | i,  and every other
+// pair no key.  The expert rows order the pairs by (partition, expert, token,
+// slot), i.e. by K, so
+//   exp_row[t, k]     = #{ valid i : K_i < K_(t,k) }
+//   expert_offset[e]  = #{ valid i : K_i < (p(e) * G + e) << 13 }
+//                     = sum of the counts of the experts before e in
+//                       (partition, id) order (experts placed nowhere last)
+//   part_offset[p]    = sum of the counts of the experts on partitions < p
+// and with dedup, token masks m_t (bit p: t holds an expert on p) give
+//   disp_row[t, p]    = sum over t' of popc(m_t' & (2^p - 1))
+//                       + #{ t' < t : bit p of m_t' }     (bit p of m_t set)
+//   part_offset[p]    = sum over t' of popc(m_t' & (2^p - 1)).
+// A block therefore needs no scan and no expert order for its own rows: it
+// counts.
+//
+// Block (b, y) of 512 threads owns tokens [t0, t0 + nt), t0 = b * T, T =
+// ceil(M / 148) (about one block per SM), and slice y of their flat 16-byte
+// units:
+//   1. issues the loads of its units of x[t0 .. t0 + nt) (contiguous rows)
+//      so they are in flight while the layout is computed;
 //   2. stages every routing id and the placement map in shared memory;
-//      warp 0 orders the experts by (partition, id) meanwhile;
-//   3. counts, per expert, the valid pairs before t0 and from t0 on (with
-//      dedup also, per partition, the tokens before t0 and from t0 on);
-//   4. scans the expert totals in that order (warp 0) and the partition
-//      sizes (warp 1);
-//   5. warp 0 walks the chunk's tokens in order with running counters:
-//        exp_row[t,k]  = expert_offset[e] + (pairs of e before t)
-//                        + (slots k' < k of t with the same expert)
-//        disp_row[t,p] = part_offset[p] + (tokens before t holding p)
-//   6. copies (bf16) or quantises and copies (fp8) its vectors to the rows;
-//   7. if asked, writes its share of the grouped-GEMM tile metadata (warp 1
-//      scanned the tiles per expert during step 5).
-// Every index is the one the tiled layout gives (stable (partition, expert,
-// token, slot) order, dedup rows in (partition, token) order), so results are
-// bit-identical to moe_layout followed by moe_dispatch.  Block (0, 0) writes
-// the counts, offsets and status word; blocks with y = 0 write their chunk's
-// index entries.  Work per block grows with M * topk, so the schedule is
-// taken only up to MOE_FUSED_ITEMS routed pairs.
+//   3. computes every pair's key, the expert histogram of the valid pairs,
+//      the invalid-input flags and, with dedup, every token's mask;
+//   4. answers rank queries, one warp per query: the rows of its own pairs
+//      (and dedup rows of its own tokens), and -- blocks with y = 0 -- its
+//      share of the per-expert and per-partition outputs (expert e and
+//      partition p go to block e mod gridDim.x and p mod gridDim.x), from the
+//      histogram; block (0, 0) also the totals and the status word.  With
+//      tile metadata requested, the owner of an expert also counts the tiles
+//      of the experts before it (tile_first[e]) and writes the expert's
+//      tiles;
+//   5. (y = 0) writes its pairs' index entries, then every block copies (bf16)
+//      or quantises once and copies (fp8) its units to every row of their
+//      token, reading the rows from shared memory.
+// Three block barriers in all.  Every index equals the one the tiled layout
+// gives (the same stable order, the same dedup rows), so results are
+// bit-identical to moe_layout followed by moe_dispatch.  Work per block grows
+// with M * topk (every block reads every id once per query), so the schedule
+// is taken only up to MOE_FUSED_ITEMS routed pairs.
 #include <algorithm>
 
 #include "fp8_device.cuh"
@@ -48,11 +63,17 @@ namespace moe {
 namespace {
 
 constexpr int kFThreads = 512;
-constexpr int kMaxFusedItems = 8192;  // the shared-memory plan holds at most this many ids
-constexpr int kMaxChunk = 16;         // tokens per block
-constexpr int kSMs = 148;
+constexpr int kFWarps = kFThreads / kWarp;
+constexpr int kIdxBits = 13;                   // pair index field of the sort key
+constexpr int kMaxFusedItems = 1 << kIdxBits;  // so at most this many pairs
 static_assert(MOE_FUSED_ITEMS >= 1 && MOE_FUSED_ITEMS <= kMaxFusedItems, "fused batch limit");
-constexpr int kMaxDest = MOE_MAX_E_PART > MOE_MAX_TOPK ? MOE_MAX_E_PART : MOE_MAX_TOPK;
+// (partition * G + expert) for partitions 0..E_part (E_part: placed nowhere)
+static_assert(((long long)(MOE_MAX_E_PART + 1) * MOE_MAX_G << kIdxBits) <= 0xffffffffLL,
+              "sort key width");
+constexpr unsigned kNoKey = 0xffffffffu;  // pair left out: above every key
+constexpr int kMaxChunk = 16;             // tokens per block
+constexpr int kSMs = 148;
+constexpr int kExpertsPerBlock = 16;      // blocks added so that none owns more experts
 
 __host__ __device__ constexpr int up4(int x) { return (x + 3) & ~3; }
 
@@ -60,6 +81,7 @@ struct FusedArgs {
   int M, G, topk, E, dedup;
   int N8;   // 16-byte chunks per bf16 row (N / 8)
   int T;    // tokens per block
+  int nb;   // blocks with tokens (blocks [nb, gridDim.x) only write per-expert outputs)
   const int* __restrict__ idx;      // [M][topk]
   const int* __restrict__ part_of;  // [G]
   const uint4* __restrict__ x;      // [M][N8]
@@ -79,28 +101,30 @@ struct FusedArgs {
 
 // shared-memory plan in ints, every array 16-byte aligned
 struct FusedSmem {
-  int ids, part_s, hb, ha, pos, scan, tscan, order, kcnt, pb, pa, poff, prow, dst, nd, misc, total;
-  __host__ __device__ FusedSmem(int n_items, int G, int E) {
+  int ids, keys, part_s, hist, masks, rows, drows, misc, total;
+  __host__ __device__ FusedSmem(int n_items, int M, int G, int E, int T, int topk, int dedup) {
     int o = 0;
-    ids = o; o += up4(n_items);   // every routing id
-    part_s = o; o += up4(G);      // placement map
-    hb = o; o += up4(G);          // per expert: valid pairs before the current token
-    ha = o; o += up4(G);          // ... from t0 on, then the expert's total
-    pos = o; o += up4(G);         // expert -> position in (partition, id) order
-    scan = o; o += up4(G);        // expert totals in that order -> exclusive scan
-    tscan = o; o += up4(G);       // tiles: first tile per expert in that order
-    order = o; o += up4(G);       // tiles: expert at each position of that order
-    kcnt = o; o += up4(E + 1);    // scratch of the expert order
-    pb = o; o += up4(E);          // dedup: tokens before the current token holding p
-    pa = o; o += up4(E);          // ... from t0 on (without dedup: rows); then the total
-    poff = o; o += up4(E + 1);    // partition offsets
-    prow = o; o += up4(E);        // dedup: the current token's row per partition (-1: none)
-    dst = o; o += kMaxChunk * kMaxDest;  // destination rows of each chunk token
-    nd = o; o += kMaxChunk;              // ... and their number
-    misc = o; o += 4;             // [bad expert, bad placement, R_exp, number of tiles]
+    ids = o; o += up4(n_items);                 // every routing id
+    keys = o; o += up4(n_items);                // every pair's sort key
+    part_s = o; o += up4(G);                    // placement map
+    hist = o; o += up4(G);                      // valid pairs per expert
+    masks = o; o += dedup ? 2 * up4(M) : 0;     // dedup: partition mask of every token (u64)
+    rows = o; o += up4(T * topk);               // expert row of each pair of the chunk
+    drows = o; o += dedup ? up4(T * E) : 0;     // dedup: row of each (chunk token, partition)
+    misc = o; o += 4;                           // [invalid-input flags]
     total = o;
   }
 };
+
+// Warp-wide sum (every lane gets it).
+__device__ __forceinline__ int warp_sum(int v) { return __reduce_add_sync(kFull, v); }
+
+// (partition * G + e): the expert's place in (partition, id) order, experts
+// placed nowhere last.
+__device__ __forceinline__ int expert_rank_key(const int* part_s, int G, int E, int e) {
+  const int p = part_s[e];
+  return (valid_part(p, E) ? p : E) * G + e;
+}
 
 // Units: bf16 16-byte chunks, or fp8 16-column groups (two chunks, one lane
 // of an 8-lane scale block).  Block (b, y) owns flat units
@@ -109,25 +133,25 @@ template <bool FP8, int U>
 __global__ void __launch_bounds__(kFThreads, 1) layout_dispatch_kernel(FusedArgs a) {
   extern __shared__ __align__(16) int sm[];
   const int n_items = a.M * a.topk;
-  const FusedSmem P(n_items, a.G, a.E);
+  const FusedSmem P(n_items, a.M, a.G, a.E, a.T, a.topk, a.dedup);
   int* ids = sm + P.ids;
+  unsigned* keys = reinterpret_cast<unsigned*>(sm + P.keys);
   int* part_s = sm + P.part_s;
-  int* hb = sm + P.hb;
-  int* ha = sm + P.ha;
-  int* pos = sm + P.pos;
-  int* scan = sm + P.scan;
-  int* pb = sm + P.pb;
-  int* pa = sm + P.pa;
-  int* poff = sm + P.poff;
+  int* hist = sm + P.hist;
+  unsigned long long* masks = reinterpret_cast<unsigned long long*>(sm + P.masks);
+  int* rows = sm + P.rows;
+  int* drows = sm + P.drows;
   int* misc = sm + P.misc;
-  const int tid = threadIdx.x;
-  const int G = a.G, E = a.E, topk = a.topk;
-  const int t0 = blockIdx.x * a.T;
-  const int nt = min(a.T, a.M - t0);
-  const int i0 = t0 * topk;  // first routed pair of the chunk
+  const int tid = threadIdx.x, lane = lane_id(), warp = warp_id();
+  const int G = a.G, E = a.E, topk = a.topk, M = a.M;
+  const int bx = blockIdx.x, nbx = gridDim.x;
   const bool writer = blockIdx.y == 0;
+  const int t0 = bx * a.T;
+  const int nt = bx < a.nb ? min(a.T, M - t0) : 0;
+  const int i0 = t0 * topk;  // first routed pair of the chunk
   pdl_wait();
   pdl_trigger();
+  if (nt == 0 && !writer) return;  // an expert-only column past the first slice: no work
 
   // 1. this block's units of the chunk, in flight while the layout is computed
   const int units = FP8 ? (a.N8 >> 1) : a.N8;
@@ -150,191 +174,186 @@ __global__ void __launch_bounds__(kFThreads, 1) layout_dispatch_kernel(FusedArgs
     }
   }
 
-  // 2. warp 0: the placement map and the expert order (which needs nothing
-  // else); warps 1..: the routing ids and the zeroed counters
-  if (warp_id() == 0) {
-    for (int e = lane_id(); e < G; e += kWarp) part_s[e] = __ldg(a.part_of + e);
-    __syncwarp();
-    expert_order_warp(part_s, G, E, pos, sm + P.kcnt);
+  // 2. every routing id and the placement map; zeroed histogram and flags
+  if ((reinterpret_cast<uintptr_t>(a.idx) & 15) == 0) {
+    const int n4 = n_items >> 2;
+    const int4* s4 = reinterpret_cast<const int4*>(a.idx);
+    int4* k4 = reinterpret_cast<int4*>(ids);
+    for (int i = tid; i < n4; i += kFThreads) k4[i] = __ldg(s4 + i);
+    for (int i = (n4 << 2) + tid; i < n_items; i += kFThreads) ids[i] = __ldg(a.idx + i);
   } else {
-    constexpr int kRest = kFThreads - kWarp;
-    const int r = tid - kWarp;
-    if ((reinterpret_cast<uintptr_t>(a.idx) & 15) == 0) {
-      const int n4 = n_items >> 2;
-      const int4* s4 = reinterpret_cast<const int4*>(a.idx);
-      int4* k4 = reinterpret_cast<int4*>(ids);
-      for (int i = r; i < n4; i += kRest) k4[i] = __ldg(s4 + i);
-      for (int i = (n4 << 2) + r; i < n_items; i += kRest) ids[i] = __ldg(a.idx + i);
-    } else {
-      for (int i = r; i < n_items; i += kRest) ids[i] = __ldg(a.idx + i);
-    }
-    for (int e = r; e < G; e += kRest) {
-      hb[e] = 0;
-      ha[e] = 0;
-    }
-    for (int p = r; p < E; p += kRest) {
-      pb[p] = 0;
-      pa[p] = 0;
-    }
-    if (r < 4) misc[r] = 0;
+    for (int i = tid; i < n_items; i += kFThreads) ids[i] = __ldg(a.idx + i);
   }
+  for (int e = tid; e < G; e += kFThreads) {
+    part_s[e] = __ldg(a.part_of + e);
+    hist[e] = 0;
+  }
+  if (tid < 4) misc[tid] = 0;
   __syncthreads();
 
-  // 3. counts before / from t0; invalid input
-  bool bad = false;
+  // 3. sort keys, histogram of the valid pairs, invalid input, token masks
+  int bad = 0;
   for (int i = tid; i < n_items; i += kFThreads) {
     const int e = ids[i];
+    unsigned key = kNoKey;
     if (e >= 0 && e < G) {
-      if (valid_part(part_s[e], E)) atomicAdd(i < i0 ? &hb[e] : &ha[e], 1);
+      const int p = part_s[e];
+      if (valid_part(p, E)) {
+        key = ((unsigned)(p * G + e) << kIdxBits) | (unsigned)i;
+        atomicAdd(&hist[e], 1);
+      }
     } else {
-      bad = true;
+      bad |= MOE_STATUS_BAD_EXPERT;
     }
+    keys[i] = key;
   }
-  if (bad) atomicOr(&misc[0], 1);
-  bool badp = false;
-  for (int e = tid; e < G; e += kFThreads) badp |= !valid_part(part_s[e], E);
-  if (badp) atomicOr(&misc[1], 1);
+  for (int e = tid; e < G; e += kFThreads)
+    if (!valid_part(part_s[e], E)) bad |= MOE_STATUS_BAD_PART;
+  if (bad) atomicOr(&misc[0], bad);
   if (a.dedup) {
-    const int lane = lane_id();
-    for (int base = 0; base < a.M; base += kFThreads) {
-      const int tt = base + tid;
-      unsigned long long mask = 0ull;
-      if (tt < a.M) {
-        for (int k = 0; k < topk; ++k) {
-          const int e = ids[tt * topk + k];
-          if (e >= 0 && e < G && valid_part(part_s[e], E)) mask |= 1ull << part_s[e];
-        }
+    for (int t = tid; t < M; t += kFThreads) {
+      unsigned long long m = 0ull;
+      for (int k = 0; k < topk; ++k) {
+        const int e = ids[t * topk + k];
+        if (e >= 0 && e < G && valid_part(part_s[e], E)) m |= 1ull << part_s[e];
       }
-      const bool before = tt < t0;
-      for (int p = 0; p < E; ++p) {
-        const bool has = (mask >> p) & 1ull;
-        const unsigned bb = __ballot_sync(kFull, has && before);
-        const unsigned ba = __ballot_sync(kFull, has && !before);
-        if (lane == 0) {
-          if (bb) atomicAdd(&pb[p], __popc(bb));
-          if (ba) atomicAdd(&pa[p], __popc(ba));
-        }
-      }
+      masks[t] = m;
     }
   }
   __syncthreads();
 
-  // 4. expert totals (into ha) in (partition, id) order; rows per partition
-  for (int e = tid; e < G; e += kFThreads) {
-    const int tot = hb[e] + ha[e];
-    ha[e] = tot;
-    scan[pos[e]] = tot;
-    if (!a.dedup && tot && valid_part(part_s[e], E)) atomicAdd(&pa[part_s[e]], tot);
-  }
-  __syncthreads();
-  if (warp_id() == 0) {
-    const int R_exp = warp_exclusive_scan(scan, G);
-    if (lane_id() == 0) misc[2] = R_exp;
-  } else if (warp_id() == 1) {  // partition totals (into pa) and offsets
-    for (int p = lane_id(); p < E; p += kWarp) {
-      const int tot = pb[p] + pa[p];
-      pa[p] = tot;
-      poff[p] = tot;
-    }
-    __syncwarp();
-    const int R_disp = warp_exclusive_scan(poff, E);
-    if (lane_id() == 0) poff[E] = R_disp;
-  }
-  __syncthreads();
-
-  // 5. the chunk's rows, token by token (warp 0; hb and pb become running
-  // counters); the tiles per expert (warp 1); the batch's counts and offsets
-  // (block (0, 0))
-  if (warp_id() == 1 && a.tiles.block_m > 0) {
-    const int n = tiles_scan_warp(pos, G, a.tiles.block_m, [&](int e) { return ha[e]; },
-                                  sm + P.tscan, sm + P.order);
-    if (lane_id() == 0) misc[3] = n;
-  }
-  if (warp_id() == 0) {
-    int* prow = sm + P.prow;
-    const int lane = lane_id();
-    const unsigned lt = lanemask_lt();
-    for (int j = 0; j < nt; ++j) {
+  // 4. rank queries, one warp each: [own pairs | own dedup (token, partition)
+  // | owned experts | owned partitions | totals (block (0, 0))]
+  const int n_pair = nt * topk;
+  const int n_dd = a.dedup ? nt * E : 0;
+  const int n_exp = writer && bx < G ? (G - bx + nbx - 1) / nbx : 0;
+  const int n_prt = writer && bx < E ? (E - bx + nbx - 1) / nbx : 0;
+  const int n_tot = writer && bx == 0 ? 1 : 0;
+  const int q_dd = n_pair, q_exp = q_dd + n_dd, q_prt = q_exp + n_exp, q_tot = q_prt + n_prt;
+  const int nq = q_tot + n_tot;
+  const int bm = a.tiles.block_m;
+  for (int q = warp; q < nq; q += kFWarps) {
+    if (q < q_dd) {  // expert row of pair i0 + q
+      const unsigned kj = keys[i0 + q];
+      int r = -1;
+      if (kj != kNoKey) {
+        int c = 0;
+        for (int i = lane; i < n_items; i += kWarp) c += keys[i] < kj;
+        r = warp_sum(c);
+      }
+      if (lane == 0) rows[q] = r;
+    } else if (q < q_exp) {  // dedup row of (token t0 + j, partition p)
+      const int j = (q - q_dd) / E, p = (q - q_dd) - j * E;
       const int t = t0 + j;
-      const int* tid_ids = ids + t * topk;
-      int* dst = sm + P.dst + j * kMaxDest;
-      int nd = 0;
-      if (a.dedup) {  // one row per partition holding any of t's experts, in partition order
-        for (int base = 0; base < E; base += kWarp) {
-          const int p = base + lane;
-          bool has = false;
-          if (p < E) {
-            for (int k = 0; k < topk; ++k) {
-              const int e = tid_ids[k];
-              has |= e >= 0 && e < G && part_s[e] == p;
-            }
-            const int row = has ? poff[p] + pb[p] : -1;
-            prow[p] = row;
-            pb[p] += has;
-            if (writer) {
-              a.disp_row[(size_t)t * E + p] = row;
-              if (has) a.disp_token[row] = t;
-            }
-          }
-          const unsigned bal = __ballot_sync(kFull, has);
-          if (has) dst[nd + __popc(bal & lt)] = prow[p];
-          nd += __popc(bal);
+      int r = -1;
+      if ((masks[t] >> p) & 1ull) {
+        const unsigned long long below = (1ull << p) - 1ull;  // p <= 63
+        int c = 0;
+        for (int u = lane; u < M; u += kWarp) {
+          const unsigned long long m = masks[u];
+          c += __popcll(m & below) + (u < t ? (int)((m >> p) & 1ull) : 0);
         }
-        __syncwarp();
+        r = warp_sum(c);
       }
-      for (int base = 0; base < topk; base += kWarp) {  // one row per valid slot
-        const int k = base + lane;
-        int row = -1, e = -1;
-        if (k < topk) {
-          e = tid_ids[k];
-          if (e >= 0 && e < G && valid_part(part_s[e], E)) {
-            int dup = 0;
-            for (int q = 0; q < k; ++q) dup += tid_ids[q] == e;
-            row = scan[pos[e]] + hb[e] + dup;
-          }
-          if (writer) {
-            a.exp_row[(size_t)t * topk + k] = row;
-            if (row >= 0) {
-              if (a.dedup)
-                a.exp_to_disp[row] = prow[part_s[e]];
-              else
-                a.disp_token[row] = t;
-            }
-          }
+      if (lane == 0) drows[j * E + p] = r;
+    } else if (q < q_prt) {  // expert e: count, first row, and its tiles
+      const int e = bx + (q - q_exp) * nbx;
+      const int ke = expert_rank_key(part_s, G, E, e);
+      int off = 0, tf = 0;
+      for (int f = lane; f < G; f += kWarp) {
+        if (expert_rank_key(part_s, G, E, f) < ke) {
+          const int c = hist[f];
+          off += c;
+          if (bm > 0) tf += c > 0 ? (c - 1) / bm + 1 : 0;
         }
-        if (!a.dedup) {
-          const unsigned bal = __ballot_sync(kFull, row >= 0);
-          if (row >= 0) dst[nd + __popc(bal & lt)] = row;
-          nd += __popc(bal);
-        }
-        __syncwarp();
-        if (row >= 0) atomicAdd(&hb[e], 1);  // after every lane of this pass has read hb
-        __syncwarp();
       }
-      if (lane == 0) sm[P.nd + j] = nd;
-      __syncwarp();
-    }
-  }
-  if (blockIdx.x == 0 && writer) {
-    for (int e = tid; e < G; e += kFThreads) {
-      a.expert_count[e] = ha[e];
-      a.expert_offset[e] = scan[pos[e]];
-    }
-    for (int p = tid; p < E; p += kFThreads) {
-      a.part_count[p] = pa[p];
-      a.part_offset[p] = poff[p];
-    }
-    if (tid == 0) {
-      a.expert_offset[G] = misc[2];
-      a.part_offset[E] = poff[E];
-      *a.status = (misc[0] ? MOE_STATUS_BAD_EXPERT : 0) | (misc[1] ? MOE_STATUS_BAD_PART : 0);
+      off = warp_sum(off);
+      const int cnt = hist[e];
+      if (lane == 0) {
+        a.expert_count[e] = cnt;
+        a.expert_offset[e] = off;
+      }
+      if (bm > 0) {
+        tf = warp_sum(tf);
+        if (lane == 0) a.tiles.tile_first[e] = tf;
+        const int nt_e = cnt > 0 ? (cnt - 1) / bm + 1 : 0;
+        for (int j = lane; j < nt_e; j += kWarp) {
+          a.tiles.tile_expert[tf + j] = e;
+          a.tiles.tile_row[tf + j] = off + j * bm;
+          a.tiles.tile_rows[tf + j] = min(bm, cnt - j * bm);
+        }
+      }
+    } else if (q < q_tot) {  // partition p: rows and first row
+      const int p = bx + (q - q_prt) * nbx;
+      int off = 0, cnt = 0;
+      if (a.dedup) {
+        const unsigned long long below = (1ull << p) - 1ull;
+        for (int u = lane; u < M; u += kWarp) {
+          const unsigned long long m = masks[u];
+          off += __popcll(m & below);
+          cnt += (int)((m >> p) & 1ull);
+        }
+      } else {
+        for (int f = lane; f < G; f += kWarp) {
+          const int pf = part_s[f];
+          if (valid_part(pf, E)) {
+            off += pf < p ? hist[f] : 0;
+            cnt += pf == p ? hist[f] : 0;
+          }
+        }
+      }
+      off = warp_sum(off);
+      cnt = warp_sum(cnt);
+      if (lane == 0) {
+        a.part_count[p] = cnt;
+        a.part_offset[p] = off;
+      }
+    } else {  // totals: R_exp, R_disp, number of tiles; the status word
+      int r_exp = 0, n_tiles = 0, r_disp = 0;
+      for (int f = lane; f < G; f += kWarp) {
+        const int c = hist[f];
+        r_exp += c;
+        if (bm > 0) n_tiles += c > 0 ? (c - 1) / bm + 1 : 0;
+      }
+      if (a.dedup)
+        for (int u = lane; u < M; u += kWarp) r_disp += __popcll(masks[u]);
+      r_exp = warp_sum(r_exp);
+      n_tiles = warp_sum(n_tiles);
+      r_disp = a.dedup ? warp_sum(r_disp) : r_exp;
+      if (lane == 0) {
+        a.expert_offset[G] = r_exp;
+        a.part_offset[E] = r_disp;
+        if (bm > 0) a.tiles.tile_first[G] = n_tiles;
+        *a.status = misc[0];
+      }
     }
   }
   __syncthreads();
 
-  // 6. copy (bf16) or quantise once and copy (fp8) each unit to its token's rows
-  const int* dst_all = sm + P.dst;
-  const int* nd_all = sm + P.nd;
+  // 5. the chunk's index entries (y = 0), then the copy to every row
+  if (writer) {
+    for (int q = tid; q < n_pair; q += kFThreads) {
+      const int r = rows[q];
+      a.exp_row[(size_t)i0 + q] = r;
+      if (r >= 0) {
+        const int j = q / topk;
+        if (a.dedup)
+          a.exp_to_disp[r] = drows[j * E + part_s[ids[i0 + q]]];
+        else
+          a.disp_token[r] = t0 + j;
+      }
+    }
+    for (int q = tid; q < n_dd; q += kFThreads) {
+      const int j = q / E, t = t0 + j;
+      const int r = drows[q];
+      a.disp_row[(size_t)t * E + (q - j * E)] = r;
+      if (r >= 0) a.disp_token[r] = t;
+    }
+  }
+  // destinations of chunk token j: its pairs' rows in slot order, or with
+  // dedup its rows in partition order (-1 entries skipped)
+  const int nd = a.dedup ? E : topk;
+  const int* dtab = a.dedup ? drows : rows;
   uint4* recv = static_cast<uint4*>(a.recv);  // rows of `units` 16-byte chunks
   if (!FP8) {
 #pragma unroll
@@ -342,8 +361,11 @@ __global__ void __launch_bounds__(kFThreads, 1) layout_dispatch_kernel(FusedArgs
       const int v = v0 + u * kFThreads;
       if (v < V) {
         const int j = v / units, c = v - j * units;
-        const int* dst = dst_all + j * kMaxDest;
-        for (int d = 0; d < nd_all[j]; ++d) st_v4(recv + (size_t)dst[d] * units + c, lo[u]);
+        const int* dst = dtab + j * nd;
+        for (int d = 0; d < nd; ++d) {
+          const int r = dst[d];
+          if (r >= 0) st_v4(recv + (size_t)r * units + c, lo[u]);
+        }
       }
     }
   } else {
@@ -356,27 +378,15 @@ __global__ void __launch_bounds__(kFThreads, 1) layout_dispatch_kernel(FusedArgs
       const int v = v0 + u * kFThreads;
       if (v < V) {
         const int j = v / units, c = v - j * units;
-        const int* dst = dst_all + j * kMaxDest;
-        for (int d = 0; d < nd_all[j]; ++d) {
-          const size_t r = (size_t)dst[d];
-          st_v4(recv + r * units + c, q);
-          if (scale_lane) a.recv_scale[r * N128 + (c >> 3)] = s;
+        const int* dst = dtab + j * nd;
+        for (int d = 0; d < nd; ++d) {
+          const int r = dst[d];
+          if (r < 0) continue;
+          st_v4(recv + (size_t)r * units + c, q);
+          if (scale_lane) a.recv_scale[(size_t)r * N128 + (c >> 3)] = s;
         }
       }
     }
-  }
-  // 7. this block's share of the tiles; block (0, 0): each expert's first tile
-  if (a.tiles.block_m > 0 && writer) {
-    const int* tscan = sm + P.tscan;
-    const int n = misc[3];
-    if (blockIdx.x == 0) {
-      for (int e = tid; e < G; e += kFThreads) a.tiles.tile_first[e] = tscan[pos[e]];
-      if (tid == 0) a.tiles.tile_first[G] = n;
-    }
-    int k0, k1;
-    tiles_share(n, blockIdx.x, gridDim.x, k0, k1);
-    tiles_write(a.tiles, tscan, sm + P.order, G, k0, k1, [&](int e) { return scan[pos[e]]; },
-                [&](int e) { return ha[e]; });
   }
 }
 
@@ -421,14 +431,17 @@ cudaError_t launch_layout_dispatch(const moe_problem_t& p, const int32_t* topk_i
   a.tiles = tiles;
 
   a.T = std::min(kMaxChunk, (p.M + kSMs - 1) / kSMs);
-  const int blocks = (p.M + a.T - 1) / a.T;
-  const size_t smem = sizeof(int) * (size_t)FusedSmem(p.M * p.topk, p.G, p.E_part).total;
+  a.nb = (p.M + a.T - 1) / a.T;
+  // enough blocks that none owns more than kExpertsPerBlock experts
+  const int nbx = std::max(a.nb, (p.G + kExpertsPerBlock - 1) / kExpertsPerBlock);
+  const size_t smem = sizeof(int) *
+      (size_t)FusedSmem(p.M * p.topk, p.M, p.G, p.E_part, a.T, p.topk, p.dedup).total;
   const int units = p.fp8 ? a.N8 / 2 : a.N8;
   const int V = a.T * units;  // units of a full chunk
   const int Umax = p.fp8 ? 4 : 8;
   const int U = std::min(Umax, (V + kFThreads - 1) / kFThreads);
   const int per_block = kFThreads * U;
-  const dim3 grid(blocks, (V + per_block - 1) / per_block);
+  const dim3 grid(nbx, (V + per_block - 1) / per_block);
   cudaError_t e;
   if (!p.fp8) {
     switch (U) {
