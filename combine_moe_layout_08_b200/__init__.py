@@ -7,6 +7,9 @@ Python face of libmoe_layout.so, with the C names:
 * :func:`moe_combine`  -- gate-weighted, slot-ordered combine
 * :func:`moe_combine_partial` / :func:`moe_combine_reduce` -- the two-level
   combine of a deduplicated dispatch (per partition, then per token)
+* :func:`moe_ep_plan` -- offsets of an expert-parallel exchange over W ranks
+  from every rank's counts; :func:`ep_all_gather_counts` gathers those counts
+  over a process group (the counts exchange itself, torch.distributed)
 
 Tensors are passed as device pointers with the current CUDA stream; this
 module checks dtypes, shapes and devices, allocates nothing inside the calls
@@ -23,7 +26,7 @@ import torch
 
 from . import _lib
 from ._lib import (MOE_MAX_E_PART, MOE_MAX_G, MOE_MAX_N, MOE_MAX_TOPK, MOE_STATIC_SCRATCH_BYTES,
-                   MOE_STATUS_BAD_EXPERT,
+                   MOE_STATUS_BAD_COUNT, MOE_STATUS_BAD_EXPERT,
                    MOE_STATUS_BAD_PART, MOE_STATUS_BAD_ROW, MoEError)
 
 __all__ = ["MoEProblem", "MoELayout", "MoEBuffers", "MoEError", "alloc_layout",
@@ -31,7 +34,8 @@ __all__ = ["MoEProblem", "MoELayout", "MoEBuffers", "MoEError", "alloc_layout",
            "moe_layout_dispatch", "moe_layout_dispatch_fused", "moe_expert_tiles",
            "expert_tiles_capacity", "alloc_expert_tiles", "ExpertTiles", "moe_combine", "moe_combine_partial", "moe_combine_reduce",
            "moe_status_string", "moe_abi_version", "MOE_STATUS_BAD_EXPERT",
-           "MOE_STATUS_BAD_PART", "MOE_STATUS_BAD_ROW", "MOE_MAX_G", "MOE_MAX_E_PART",
+           "MOE_STATUS_BAD_PART", "MOE_STATUS_BAD_ROW", "MOE_STATUS_BAD_COUNT", "MOE_MAX_G",
+           "MOE_MAX_E_PART", "EpPlan", "alloc_ep_plan", "moe_ep_plan", "ep_all_gather_counts",
            "MOE_MAX_TOPK", "MOE_MAX_N"]
 
 
@@ -328,6 +332,75 @@ def moe_combine_reduce(prob: MoEProblem, z: torch.Tensor, lay: MoELayout, out: t
                                         out.data_ptr(), _stream(z, stream))
     if rc:
         raise MoEError("moe_combine_reduce", rc)
+
+
+@dataclasses.dataclass
+class EpPlan:
+    """Device arrays of one rank's exchange plan (int32), see ``moe_ep_plan_t``."""
+    send_offset: torch.Tensor                          # [W]
+    src_offset: torch.Tensor                           # [W]
+    recv_count: torch.Tensor                           # [W]
+    recv_offset: torch.Tensor                          # [W + 1]
+    status: torch.Tensor                               # [1]
+    recv_expert_count: Optional[torch.Tensor] = None   # [G]
+    recv_block_offset: Optional[torch.Tensor] = None   # [W, G]
+
+    def struct(self) -> _lib.EpPlanStruct:
+        def p(t):
+            return None if t is None else t.data_ptr()
+        return _lib.EpPlanStruct(p(self.send_offset), p(self.src_offset), p(self.recv_count),
+                                 p(self.recv_offset), p(self.recv_expert_count),
+                                 p(self.recv_block_offset), p(self.status))
+
+
+def alloc_ep_plan(world: int, G: int = 0, device="cuda") -> EpPlan:
+    """Plan arrays for ``world`` ranks; per-expert arrays when ``G`` > 0."""
+    i32 = dict(dtype=torch.int32, device=device)
+    return EpPlan(torch.empty(world, **i32), torch.empty(world, **i32), torch.empty(world, **i32),
+                  torch.empty(world + 1, **i32), torch.empty(1, **i32),
+                  torch.empty(G, **i32) if G else None,
+                  torch.empty((world, G), **i32) if G else None)
+
+
+def moe_ep_plan(world: int, rank: int, part_counts: torch.Tensor, plan: EpPlan,
+                expert_counts: Optional[torch.Tensor] = None,
+                part_of: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Rank ``rank``'s offsets for the exchange of dispatch rows among
+    ``world`` ranks, from every rank's part_count ``part_counts`` [W, W]
+    (and, without dedup, every rank's expert_count ``expert_counts`` [W, G]
+    with the placement ``part_of`` [G]), into ``plan``."""
+    dev = part_counts.device
+    _check(part_counts, "part_counts", torch.int32, world * world, dev)
+    for name in ("send_offset", "src_offset", "recv_count"):
+        _check(getattr(plan, name), name, torch.int32, world, dev)
+    _check(plan.recv_offset, "recv_offset", torch.int32, world + 1, dev)
+    _check(plan.status, "status", torch.int32, 1, dev)
+    G = 0
+    if expert_counts is not None:
+        G = expert_counts.numel() // max(world, 1)
+        _check(expert_counts, "expert_counts", torch.int32, world * G, dev)
+        _check(part_of, "part_of", torch.int32, G, dev)
+        _check(plan.recv_expert_count, "recv_expert_count", torch.int32, G, dev)
+        _check(plan.recv_block_offset, "recv_block_offset", torch.int32, world * G, dev)
+    ps = plan.struct()
+    rc = _lib.load().moe_ep_plan(world, rank, G, part_counts.data_ptr(),
+                                 None if expert_counts is None else expert_counts.data_ptr(),
+                                 None if part_of is None else part_of.data_ptr(),
+                                 ctypes.byref(ps), _stream(part_counts, stream))
+    if rc:
+        raise MoEError("moe_ep_plan", rc)
+
+
+def ep_all_gather_counts(counts: torch.Tensor, group=None) -> torch.Tensor:
+    """The counts exchange: every rank's ``counts`` [K] int32 (its part_count,
+    or its expert_count), gathered over the process group into [W, K] in rank
+    order, on the device of ``counts`` (NCCL for CUDA tensors, gloo on CPU).
+    Every rank of the group must call it, with the same K."""
+    import torch.distributed as dist
+    W = dist.get_world_size(group)
+    parts = [torch.empty_like(counts) for _ in range(W)]
+    dist.all_gather(parts, counts.contiguous(), group=group)
+    return torch.stack(parts)
 
 
 class MoEBuffers:

@@ -22,6 +22,7 @@ MOE_ABI_VERSION = 1
 MOE_STATUS_BAD_EXPERT = 1
 MOE_STATUS_BAD_PART = 2
 MOE_STATUS_BAD_ROW = 4
+MOE_STATUS_BAD_COUNT = 8
 
 MOE_MAX_G = 1024
 MOE_MAX_E_PART = 64
@@ -46,6 +47,12 @@ class LayoutStruct(ctypes.Structure):
 class TilesStruct(ctypes.Structure):
     _fields_ = [("block_m", ctypes.c_int32)] + [
         (n, ctypes.c_void_p) for n in ("tile_first", "tile_expert", "tile_row", "tile_rows")]
+
+
+class EpPlanStruct(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "send_offset", "src_offset", "recv_count", "recv_offset", "recv_expert_count",
+        "recv_block_offset", "status")]
 
 
 SIGNATURES = {
@@ -79,6 +86,9 @@ SIGNATURES = {
     "moe_combine_reduce": (ctypes.c_int, [ctypes.POINTER(ProblemStruct), ctypes.c_void_p,
                                           ctypes.POINTER(LayoutStruct), ctypes.c_void_p,
                                           ctypes.c_void_p]),
+    "moe_ep_plan": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p,
+                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(EpPlanStruct),
+                                   ctypes.c_void_p]),
 }
 
 _lock = threading.Lock()

@@ -174,4 +174,21 @@ int moe_combine_reduce(const moe_problem_t* prob, const void* z, const moe_layou
                                             reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int moe_ep_plan(int32_t world, int32_t rank, int32_t G, const int32_t* part_counts,
+                const int32_t* expert_counts, const int32_t* part_of, const moe_ep_plan_t* plan,
+                moe_stream_t stream) {
+  if (world < 1 || world > MOE_MAX_E_PART || rank < 0 || rank >= world) return MOE_ERR_ARG;
+  if (!plan || !arr(part_counts)) return MOE_ERR_ARG;
+  if (!arr(plan->send_offset) || !arr(plan->src_offset) || !arr(plan->recv_count) ||
+      !arr(plan->recv_offset) || !arr(plan->status))
+    return MOE_ERR_ARG;
+  if (expert_counts) {
+    if (G < 1 || G > MOE_MAX_G || !arr(expert_counts) || !arr(part_of)) return MOE_ERR_ARG;
+    if (!arr(plan->recv_expert_count) || !arr(plan->recv_block_offset)) return MOE_ERR_ARG;
+  }
+  return cuda_rc(moe::launch_ep_plan(world, rank, expert_counts ? G : 0, part_counts,
+                                     expert_counts, part_of, *plan,
+                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

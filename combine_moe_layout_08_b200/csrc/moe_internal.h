@@ -89,6 +89,10 @@ cudaError_t launch_combine_partial(const moe_problem_t& p, const void* y, const 
 cudaError_t launch_combine_reduce(const moe_problem_t& p, const void* z, const moe_layout_t& lay,
                                   void* out, cudaStream_t stream);
 
+cudaError_t launch_ep_plan(int world, int rank, int G, const int32_t* part_counts,
+                           const int32_t* expert_counts, const int32_t* part_of,
+                           const moe_ep_plan_t& plan, cudaStream_t stream);
+
 cudaError_t launch_combine(const moe_problem_t& p, const void* y,
                            const float* w, const moe_layout_t& lay, void* out,
                            cudaStream_t stream);

@@ -53,6 +53,9 @@ typedef struct CUstream_st *moe_stream_t;
                                    pairs are left out                                   */
 #define MOE_STATUS_BAD_ROW 4    /* dispatch / combine met a row index outside the
                                    receive capacity M*topk: that copy / term skipped    */
+#define MOE_STATUS_BAD_COUNT 8  /* moe_ep_plan: a count negative, an offset past
+                                   INT32_MAX (written as -1) or expert counts that do
+                                   not add up to the partition count                    */
 
 /* limits checked by every entry point */
 #define MOE_MAX_G 1024
@@ -312,6 +315,59 @@ int moe_combine_partial(const moe_problem_t *prob, const void *y,
                         void *z, moe_stream_t stream);
 int moe_combine_reduce(const moe_problem_t *prob, const void *z,
                        const moe_layout_t *lay, void *out, moe_stream_t stream);
+
+/*
+ * Expert-parallel exchange plan.  With the partitions on W ranks (E_part = W,
+ * partition p = rank p), each rank's layout counts what it sends to every
+ * rank; an all-gather of those counts (the split_send_buf -> split_recv_buf
+ * exchange and send_split_cumsum of the Triton-distributed issue #117
+ * all-to-all) gives every rank the matrix P[s][d] of the rows source s sends
+ * to destination d.  This call turns that matrix into rank r's offsets for the
+ * data exchange into Purlin's transposed-V layout (section 3.1: destination r
+ * holds partition r of every source, in source-rank order):
+ *   world, rank    W (1..MOE_MAX_E_PART) and r (0..W-1)
+ *   part_counts    [W][W] int32, row s = the part_count of rank s's layout
+ *   expert_counts  [W][G] int32, row s = the expert_count of rank s's layout,
+ *                  or NULL.  Only without dedup, where dispatch rows are
+ *                  expert rows.
+ *   part_of        [G] int32 placement (expert -> rank); with expert_counts
+ *   G              experts (1..MOE_MAX_G); ignored without expert_counts
+ *   plan           device arrays, caller-allocated:
+ *     send_offset  [W]    sum_{s<r} P[s][d]: where r's rows for d start in d's
+ *                         receive buffer (a push, by peer stores)
+ *     src_offset   [W]    sum_{d<r} P[s][d]: where s's rows for r start in s's
+ *                         dispatch buffer (a pull, by peer loads)
+ *     recv_count   [W]    P[s][r]
+ *     recv_offset  [W+1]  sum_{s'<s} P[s'][r]: where s's rows land in r's
+ *                         receive buffer; [W] = rows r receives
+ *     recv_expert_count [G]    (with expert_counts) rows r receives per expert:
+ *                              sum_s X[s][e] for the experts on r, else 0
+ *     recv_block_offset [W][G] (with expert_counts) first row of the block of
+ *                              source s's rows of expert e in r's receive
+ *                              buffer, for the experts on r (-1 elsewhere):
+ *                              recv_offset[s] + sum of X[s][f] over the experts
+ *                              f < e on r.  The (source, expert) blocks a
+ *                              grouped GEMM over the receive buffer consumes.
+ *     status       [1]    0 or MOE_STATUS_BAD_COUNT
+ * Sums are exact in 64 bits; an offset past INT32_MAX is written as -1 and
+ * flagged.  One small kernel on `stream`; it reads only the given arrays.
+ * MOE_ERR_ARG for world, rank or G out of range and null or misaligned arrays.
+ * The data exchange itself (peer stores or loads over NVLink, or an NCCL
+ * all-to-all with these counts) is the caller's.
+ */
+typedef struct moe_ep_plan {
+    int32_t *send_offset;
+    int32_t *src_offset;
+    int32_t *recv_count;
+    int32_t *recv_offset;
+    int32_t *recv_expert_count;
+    int32_t *recv_block_offset;
+    int32_t *status;
+} moe_ep_plan_t;
+
+int moe_ep_plan(int32_t world, int32_t rank, int32_t G, const int32_t *part_counts,
+                const int32_t *expert_counts, const int32_t *part_of,
+                const moe_ep_plan_t *plan, moe_stream_t stream);
 
 #ifdef __cplusplus
 }

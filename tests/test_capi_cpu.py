@@ -234,6 +234,27 @@ def test_python_binding_fails_loudly_without_library(monkeypatch, tmp_path):
         _lib.load()
 
 
+@no_gpu
+def test_ep_plan_rejects_bad_arguments(L):
+    def plan(**over):
+        f = {n: FAKE + 4096 * (i + 1) for i, (n, _) in enumerate(_lib.EpPlanStruct._fields_)}
+        f.update(over)
+        return ctypes.byref(_lib.EpPlanStruct(**f))
+    ok = plan()
+    for world, rank in ((0, 0), (65, 0), (4, 4), (4, -1)):
+        assert L.moe_ep_plan(world, rank, 8, FAKE, None, None, ok, None) == 1
+    assert L.moe_ep_plan(4, 0, 8, None, None, None, ok, None) == 1             # no counts
+    assert L.moe_ep_plan(4, 0, 8, FAKE + 2, None, None, ok, None) == 1         # misaligned
+    assert L.moe_ep_plan(4, 0, 8, FAKE, None, None, None, None) == 1           # no plan
+    assert L.moe_ep_plan(4, 0, 8, FAKE, None, None, plan(status=None), None) == 1
+    assert L.moe_ep_plan(4, 0, 8, FAKE, None, None, plan(recv_offset=FAKE + 1), None) == 1
+    # with expert counts: G in range, placement and per-expert arrays required
+    assert L.moe_ep_plan(4, 0, 0, FAKE, FAKE, FAKE, ok, None) == 1
+    assert L.moe_ep_plan(4, 0, 1025, FAKE, FAKE, FAKE, ok, None) == 1
+    assert L.moe_ep_plan(4, 0, 8, FAKE, FAKE, None, ok, None) == 1
+    assert L.moe_ep_plan(4, 0, 8, FAKE, FAKE, FAKE, plan(recv_block_offset=None), None) == 1
+
+
 C_HOST = r"""
 #include <stdio.h>
 #include "moe_layout.h"
@@ -252,7 +273,12 @@ int main(void) {
     if (moe_layout(&bad, 0, 0, &lay, 0, 0, 0) != MOE_ERR_ARG) return 6;
     if (moe_expert_tiles(&p, 0, &lay, &tiles, 0) != MOE_ERR_ARG) return 7;
     (void)moe_layout_static; (void)moe_dispatch; (void)moe_combine;
-    (void)moe_combine_partial; (void)moe_combine_reduce;
+    (void)moe_combine_partial; (void)moe_combine_reduce; (void)moe_ep_plan;
+    {
+        moe_ep_plan_t plan = {0};
+        /* an invalid call fails on the host: rank outside [0, world) */
+        if (moe_ep_plan(2, 2, 8, 0, 0, 0, &plan, 0) != MOE_ERR_ARG) return 8;
+    }
     printf("ok\n");
     return 0;
 }
@@ -293,5 +319,6 @@ def test_python_constants_match_the_header():
     src = open(HEADER).read()
     defs = {k: v.strip() for k, v in re.findall(r"#define (MOE_\w+)[ \t]+([^/\n]+)", src)}
     for name in ("MOE_MAX_G", "MOE_MAX_E_PART", "MOE_MAX_TOPK", "MOE_MAX_N", "MOE_STATUS_BAD_EXPERT",
-                 "MOE_STATUS_BAD_PART", "MOE_STATUS_BAD_ROW", "MOE_ABI_VERSION"):
+                 "MOE_STATUS_BAD_PART", "MOE_STATUS_BAD_ROW", "MOE_STATUS_BAD_COUNT",
+                 "MOE_ABI_VERSION"):
         assert eval(defs[name]) == getattr(_lib, name), (name, defs[name])   # integer literals
