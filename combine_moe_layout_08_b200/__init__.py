@@ -10,6 +10,10 @@ Python face of libmoe_layout.so, with the C names:
 * :func:`moe_ep_plan` -- offsets of an expert-parallel exchange over W ranks
   from every rank's counts; :func:`ep_all_gather_counts` gathers those counts
   over a process group (the counts exchange itself, torch.distributed)
+* :func:`moe_ep_dispatch` / :func:`moe_ep_combine` /
+  :func:`moe_ep_combine_reduce` -- the expert-parallel data plane: rows pushed
+  into, and outputs pulled from, every rank's buffers through a table of
+  device pointers (:class:`EpPeers`)
 
 Tensors are passed as device pointers with the current CUDA stream; this
 module checks dtypes, shapes and devices, allocates nothing inside the calls
@@ -36,6 +40,7 @@ __all__ = ["MoEProblem", "MoELayout", "MoEBuffers", "MoEError", "alloc_layout",
            "moe_status_string", "moe_abi_version", "MOE_STATUS_BAD_EXPERT",
            "MOE_STATUS_BAD_PART", "MOE_STATUS_BAD_ROW", "MOE_STATUS_BAD_COUNT", "MOE_MAX_G",
            "MOE_MAX_E_PART", "EpPlan", "alloc_ep_plan", "moe_ep_plan", "ep_all_gather_counts",
+           "EpPeers", "ep_peers", "moe_ep_dispatch", "moe_ep_combine", "moe_ep_combine_reduce",
            "MOE_MAX_TOPK", "MOE_MAX_N"]
 
 
@@ -401,6 +406,91 @@ def ep_all_gather_counts(counts: torch.Tensor, group=None) -> torch.Tensor:
     parts = [torch.empty_like(counts) for _ in range(W)]
     dist.all_gather(parts, counts.contiguous(), group=group)
     return torch.stack(parts)
+
+
+@dataclasses.dataclass
+class EpPeers:
+    """Every rank's buffer as this GPU addresses it, for the expert-parallel
+    data plane: a device array of pointers (``table``, int64 [W]), optional
+    scale pointers (fp8 dispatch) and the rows each buffer holds.  ``keep``
+    holds the tensors the pointers come from, if any, so they stay alive."""
+    table: torch.Tensor
+    capacity: int
+    scale_table: Optional[torch.Tensor] = None
+    keep: tuple = ()
+
+    def struct(self) -> _lib.EpPeersStruct:
+        return _lib.EpPeersStruct(self.table.data_ptr(),
+                                  None if self.scale_table is None else self.scale_table.data_ptr(),
+                                  self.capacity)
+
+
+def ep_peers(rows, capacity: int, scales=None, device="cuda") -> EpPeers:
+    """Pointer table from per-rank buffers: tensors on this GPU (local, or
+    opened from a peer's memory handle) or raw device addresses (ints), in
+    rank order.  Building it copies W pointers to the device once; reuse it
+    across steps."""
+    def addr(t):
+        return int(t) if isinstance(t, int) else t.data_ptr()
+    table = torch.tensor([addr(t) for t in rows], dtype=torch.int64).to(device)
+    st = None if scales is None else \
+        torch.tensor([addr(t) for t in scales], dtype=torch.int64).to(device)
+    keep = tuple(t for t in list(rows) + list(scales or []) if isinstance(t, torch.Tensor))
+    return EpPeers(table, int(capacity), st, keep)
+
+
+def moe_ep_dispatch(prob: MoEProblem, x: torch.Tensor, lay: MoELayout, send_offset: torch.Tensor,
+                    peers: EpPeers, stream=None) -> None:
+    """Push dispatch: every token row of ``x`` stored into each destination
+    rank's receive buffer at this rank's ``send_offset`` (from moe_ep_plan)."""
+    dev = x.device
+    _check(x, "x", torch.bfloat16, prob.M * prob.N, dev)
+    _check(send_offset, "send_offset", torch.int32, prob.E_part, dev)
+    _check_layout(prob, lay, dev)
+    if peers.table.numel() != prob.E_part or (prob.fp8 and peers.scale_table is None):
+        raise ValueError("peers: one buffer (and with fp8 one scale buffer) per partition")
+    s, l, ps = prob.struct(), lay.struct(), peers.struct()
+    rc = _lib.load().moe_ep_dispatch(ctypes.byref(s), x.data_ptr(), ctypes.byref(l),
+                                     send_offset.data_ptr(), ctypes.byref(ps), _stream(x, stream))
+    if rc:
+        raise MoEError("moe_ep_dispatch", rc)
+
+
+def moe_ep_combine(prob: MoEProblem, y_peers: EpPeers, topk_weights: torch.Tensor, lay: MoELayout,
+                   send_offset: torch.Tensor, out: torch.Tensor, stream=None) -> None:
+    """Pull combine (no dedup): expert outputs gathered from every rank's
+    buffer and summed in slot order into ``out`` [M, N] bf16."""
+    dev = out.device
+    _check(topk_weights, "topk_weights", torch.float32, prob.M * prob.topk, dev)
+    _check(out, "out", torch.bfloat16, prob.M * prob.N, dev)
+    _check(send_offset, "send_offset", torch.int32, prob.E_part, dev)
+    _check_layout(prob, lay, dev)
+    if prob.dedup or y_peers.table.numel() != prob.E_part:
+        raise ValueError("moe_ep_combine needs a layout without dedup and one buffer per partition")
+    s, l, ps = prob.struct(), lay.struct(), y_peers.struct()
+    rc = _lib.load().moe_ep_combine(ctypes.byref(s), ctypes.byref(ps), topk_weights.data_ptr(),
+                                    ctypes.byref(l), send_offset.data_ptr(), out.data_ptr(),
+                                    _stream(out, stream))
+    if rc:
+        raise MoEError("moe_ep_combine", rc)
+
+
+def moe_ep_combine_reduce(prob: MoEProblem, z_peers: EpPeers, lay: MoELayout,
+                          send_offset: torch.Tensor, out: torch.Tensor, stream=None) -> None:
+    """Pull token-side sum of the two-level combine (dedup): each token's
+    partition rows gathered from every rank's buffer, summed in partition order."""
+    dev = out.device
+    _check(out, "out", torch.bfloat16, prob.M * prob.N, dev)
+    _check(send_offset, "send_offset", torch.int32, prob.E_part, dev)
+    _check_layout(prob, lay, dev)
+    if not prob.dedup or z_peers.table.numel() != prob.E_part:
+        raise ValueError("moe_ep_combine_reduce needs a dedup layout and one buffer per partition")
+    s, l, ps = prob.struct(), lay.struct(), z_peers.struct()
+    rc = _lib.load().moe_ep_combine_reduce(ctypes.byref(s), ctypes.byref(ps), ctypes.byref(l),
+                                           send_offset.data_ptr(), out.data_ptr(),
+                                           _stream(out, stream))
+    if rc:
+        raise MoEError("moe_ep_combine_reduce", rc)
 
 
 class MoEBuffers:

@@ -55,6 +55,10 @@ class EpPlanStruct(ctypes.Structure):
         "recv_block_offset", "status")]
 
 
+class EpPeersStruct(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("capacity", ctypes.c_int32)]
+
+
 SIGNATURES = {
     "moe_abi_version": (ctypes.c_int, []),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -86,6 +90,16 @@ SIGNATURES = {
     "moe_combine_reduce": (ctypes.c_int, [ctypes.POINTER(ProblemStruct), ctypes.c_void_p,
                                           ctypes.POINTER(LayoutStruct), ctypes.c_void_p,
                                           ctypes.c_void_p]),
+    "moe_ep_dispatch": (ctypes.c_int, [ctypes.POINTER(ProblemStruct), ctypes.c_void_p,
+                                       ctypes.POINTER(LayoutStruct), ctypes.c_void_p,
+                                       ctypes.POINTER(EpPeersStruct), ctypes.c_void_p]),
+    "moe_ep_combine": (ctypes.c_int, [ctypes.POINTER(ProblemStruct), ctypes.POINTER(EpPeersStruct),
+                                      ctypes.c_void_p, ctypes.POINTER(LayoutStruct), ctypes.c_void_p,
+                                      ctypes.c_void_p, ctypes.c_void_p]),
+    "moe_ep_combine_reduce": (ctypes.c_int, [ctypes.POINTER(ProblemStruct),
+                                             ctypes.POINTER(EpPeersStruct),
+                                             ctypes.POINTER(LayoutStruct), ctypes.c_void_p,
+                                             ctypes.c_void_p, ctypes.c_void_p]),
     "moe_ep_plan": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p,
                                    ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(EpPlanStruct),
                                    ctypes.c_void_p]),

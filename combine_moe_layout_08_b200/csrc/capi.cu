@@ -191,4 +191,42 @@ int moe_ep_plan(int32_t world, int32_t rank, int32_t G, const int32_t* part_coun
                                      reinterpret_cast<cudaStream_t>(stream)));
 }
 
+// the pointer array and its capacity (the pointers themselves are device
+// data, checked by the kernels)
+static bool valid_peers(const moe_problem_t* p, const moe_ep_peers_t* peers, bool scales) {
+  if (!peers || !peers->rows || !aligned(peers->rows, 8) || peers->capacity < 0) return false;
+  if (scales && (!peers->scales || !aligned(peers->scales, 8))) return false;
+  (void)p;
+  return true;
+}
+
+int moe_ep_dispatch(const moe_problem_t* prob, const void* x, const moe_layout_t* lay,
+                    const int32_t* send_offset, const moe_ep_peers_t* peers, moe_stream_t stream) {
+  if (!valid_problem(prob) || !valid_layout(prob, lay) || !arr(send_offset)) return MOE_ERR_ARG;
+  if (!valid_peers(prob, peers, prob->fp8 != 0)) return MOE_ERR_ARG;
+  if (prob->M > 0 && (!x || !aligned(x, 16))) return MOE_ERR_ARG;
+  return cuda_rc(moe::launch_ep_dispatch(*prob, x, *lay, send_offset, *peers,
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int moe_ep_combine(const moe_problem_t* prob, const moe_ep_peers_t* y_peers,
+                   const float* topk_weights, const moe_layout_t* lay, const int32_t* send_offset,
+                   void* out, moe_stream_t stream) {
+  if (!valid_problem(prob) || !valid_layout(prob, lay) || prob->dedup) return MOE_ERR_ARG;
+  if (!arr(send_offset) || !valid_peers(prob, y_peers, false)) return MOE_ERR_ARG;
+  if (prob->M > 0 && (!out || !aligned(out, 16) || !arr(topk_weights))) return MOE_ERR_ARG;
+  return cuda_rc(moe::launch_ep_combine(*prob, *y_peers, topk_weights, *lay, send_offset, out,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int moe_ep_combine_reduce(const moe_problem_t* prob, const moe_ep_peers_t* z_peers,
+                          const moe_layout_t* lay, const int32_t* send_offset, void* out,
+                          moe_stream_t stream) {
+  if (!valid_problem(prob) || !valid_layout(prob, lay) || !prob->dedup) return MOE_ERR_ARG;
+  if (!arr(send_offset) || !valid_peers(prob, z_peers, false)) return MOE_ERR_ARG;
+  if (prob->M > 0 && (!out || !aligned(out, 16))) return MOE_ERR_ARG;
+  return cuda_rc(moe::launch_ep_reduce(*prob, *z_peers, *lay, send_offset, out,
+                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -93,6 +93,16 @@ cudaError_t launch_ep_plan(int world, int rank, int G, const int32_t* part_count
                            const int32_t* expert_counts, const int32_t* part_of,
                            const moe_ep_plan_t& plan, cudaStream_t stream);
 
+cudaError_t launch_ep_dispatch(const moe_problem_t& p, const void* x, const moe_layout_t& lay,
+                               const int32_t* send_offset, const moe_ep_peers_t& peers,
+                               cudaStream_t stream);
+cudaError_t launch_ep_combine(const moe_problem_t& p, const moe_ep_peers_t& y, const float* w,
+                              const moe_layout_t& lay, const int32_t* send_offset, void* out,
+                              cudaStream_t stream);
+cudaError_t launch_ep_reduce(const moe_problem_t& p, const moe_ep_peers_t& z,
+                             const moe_layout_t& lay, const int32_t* send_offset, void* out,
+                             cudaStream_t stream);
+
 cudaError_t launch_combine(const moe_problem_t& p, const void* y,
                            const float* w, const moe_layout_t& lay, void* out,
                            cudaStream_t stream);

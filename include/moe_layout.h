@@ -369,6 +369,72 @@ int moe_ep_plan(int32_t world, int32_t rank, int32_t G, const int32_t *part_coun
                 const int32_t *expert_counts, const int32_t *part_of,
                 const moe_ep_plan_t *plan, moe_stream_t stream);
 
+/*
+ * Expert-parallel data plane: the dispatch and the combine with partition p
+ * on rank p (E_part = W ranks), each rank's buffers addressed through a
+ * device array of pointers -- peer mappings over NVLink (cudaIpc handles,
+ * symmetric memory), or plain local buffers when the ranks share one GPU.
+ * Rank r's dispatch rows of partition p (rows [part_offset[p],
+ * part_offset[p+1]) of its layout) occupy rows [send_offset[p],
+ * send_offset[p] + count) of rank p's receive buffer, in the same order:
+ * Purlin's transposed-V layout (section 3.1), with send_offset from rank r's
+ * moe_ep_plan.  Dispatch row r of partition p therefore lives at row
+ * send_offset[p] + r - part_offset[p] of rank p's buffers, and the outputs
+ * rank p computes in its receive order come back from the same row.
+ *   rows       [W] device array of device pointers, one per rank, each
+ *              16-byte aligned
+ *   scales     [W] device array of device pointers to fp32 scale buffers
+ *              (moe_ep_dispatch with fp8), else ignored; 4-byte aligned
+ *   capacity   rows each rank's buffer holds; rows at or past it are never
+ *              touched
+ * A row outside a rank's capacity or its partition, or a null or misaligned
+ * pointer in the array, is skipped and raises MOE_STATUS_BAD_ROW in
+ * lay->status.  The kernels never wait on another rank: the caller orders
+ * the steps (every rank's dispatch complete before any destination reads
+ * its receive buffer; every destination's outputs complete before any
+ * combine), e.g. with a barrier or an NCCL collective between them.
+ */
+typedef struct moe_ep_peers {
+    void *const *rows;
+    float *const *scales;
+    int32_t capacity;
+} moe_ep_peers_t;
+
+/*
+ * Push dispatch (Purlin section 3.2: push in the latency path; issue #117
+ * all_to_all_kernel data_src -> data_dst, scale_src -> scale_dst): each
+ * token row of x is read once and stored into every destination rank's
+ * receive buffer (peers->rows), bf16 or, with fp8, e4m3 bytes plus one
+ * scale per 128 columns into peers->scales.  The bytes of every row equal
+ * those moe_dispatch writes.  x, lay and the argument rules as moe_dispatch;
+ * send_offset [E_part] int32 (device) from moe_ep_plan.
+ */
+int moe_ep_dispatch(const moe_problem_t *prob, const void *x, const moe_layout_t *lay,
+                    const int32_t *send_offset, const moe_ep_peers_t *peers,
+                    moe_stream_t stream);
+
+/*
+ * Pull combine (prob->dedup = 0): out[t, :] = bf16( sum_k w[t,k] *
+ * y[rank p(k)][send_offset[p] + exp_row[t,k] - part_offset[p], :] ), fp32
+ * fused multiply-adds in slot order from +0 (Purlin section 3.3, SCORE), with
+ * y the ranks' expert-output buffers (y_peers->rows, bf16, rows in each
+ * rank's receive order).  Equal to moe_combine over the gathered rows.
+ */
+int moe_ep_combine(const moe_problem_t *prob, const moe_ep_peers_t *y_peers,
+                   const float *topk_weights, const moe_layout_t *lay,
+                   const int32_t *send_offset, void *out, moe_stream_t stream);
+
+/*
+ * Pull token-side sum of the two-level combine (prob->dedup = 1): out[t, :] =
+ * bf16( sum over p with disp_row[t,p] >= 0, in partition order, of
+ * z[rank p][send_offset[p] + disp_row[t,p] - part_offset[p], :] ), fp32 from
+ * +0, with z the ranks' partition-side rows (z_peers->rows, bf16, each rank's
+ * receive order).  Equal to moe_combine_reduce over the gathered rows.
+ */
+int moe_ep_combine_reduce(const moe_problem_t *prob, const moe_ep_peers_t *z_peers,
+                          const moe_layout_t *lay, const int32_t *send_offset, void *out,
+                          moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
