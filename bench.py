@@ -736,13 +736,50 @@ def run_latency_sweep(args):
                                                                  if inner else (0.0, 0.0)))
                 med.append(np.median(np.array(t), axis=0) * 1e3)
                 graph.reset()
+            # the same step without event nodes inside the graph: R x [flush,
+            # step] minus R x [flush], each timed as a whole (events outside
+            # the graphs), divided by R
+            R = 20
+            g_steps, g_flush = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_steps, stream=stream):
+                for _ in range(R):
+                    flush_w.zero_()
+                    if separate:
+                        buf.layout_(idx, po)
+                        buf.dispatch_(d["x"])
+                    else:
+                        buf.layout_dispatch_(idx, po, d["x"])
+                    buf.combine_(d["y"], gates)
+            with torch.cuda.graph(g_flush, stream=stream):
+                for _ in range(R):
+                    flush_w.zero_()
+
+            def whole(gr, n=max(10, args.steps // 10)):
+                ts = []
+                for i in range(n + 3):
+                    e0, e1 = (torch.cuda.Event(enable_timing=True) for _ in range(2))
+                    with torch.cuda.stream(stream):
+                        e0.record()
+                        gr.replay()
+                        e1.record()
+                    e1.synchronize()
+                    if i >= 3:
+                        ts.append(e0.elapsed_time(e1) * 1e3)
+                return float(np.median(ts))
+            diff = (whole(g_steps) - whole(g_flush)) / R
+            g_steps.reset()
+            g_flush.reset()
             key = "separate_" if separate else ""
+            row[key + "step_us_between_flushes"] = round(diff, 2)
             row[key + "step_us"] = round(float(med[0][0]), 2)
             row[key + "layout_dispatch_us"] = round(float(med[1][1]), 2)
             if not separate:
                 row["combine_us"] = round(float(med[1][2]), 2)
         rows.append(row)
     print(json.dumps({"metric": "decode latency against M (us, median, L2 flushed)",
+                      "note": "step_us: median of one graph replay with events at its ends; "
+                              "step_us_between_flushes: the step's share of R back-to-back "
+                              "[flush, step] replays (no event node inside the graph)",
                       "config": {"N": base.N, "G": base.G, "topk": base.topk,
                                  "E_part": base.E_part, "routing": base.routing},
                       "steps": args.steps, "rows": rows}), flush=True)

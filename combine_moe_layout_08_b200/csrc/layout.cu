@@ -29,10 +29,11 @@
 //     hardware cluster barriers.  No workspace is touched.
 //   * larger batches: about one tile per SM in two launches.
 //     layout_count_kernel writes the rows to the workspace;
-//     layout_rank_kernel stages its tile, counts it per warp and orders the
-//     experts by (partition, id) -- all from the caller's inputs, before it
-//     waits for layout_count_kernel (programmatic dependent launch) -- then
-//     reduces the rows with batched 16-byte loads from L2 and ranks its tile.
+//     layout_rank_kernel stages its tile, orders the experts by (partition,
+//     id) with every warp at once and counts its tile per warp -- all from the
+//     caller's inputs, before it waits for layout_count_kernel (programmatic
+//     dependent launch) -- then reduces the rows with batched 16-byte loads
+//     from L2 and ranks its tile.
 // In both, the tile's expert ids are cached in shared memory when they fit.
 // Asked for it, both also emit the grouped-GEMM tile metadata: one warp
 // scans the tiles per expert while the others rank, and every block writes
@@ -77,6 +78,8 @@ static_assert(kClusterItems <= kMaxCluster * kMaxTileItems, "cluster tiles must 
 // MOE_MAX_E_PART + 2, padded)
 constexpr int kRedW = 4 * kLThreads;
 static_assert(kRedW >= MOE_MAX_G + MOE_MAX_E_PART + 4, "reduction buffer narrower than a tile row");
+static_assert(2 * kRedW >= (MOE_MAX_E_PART + 1) * ((MOE_MAX_G + 31) / 32),
+              "reduction buffer smaller than the expert order's counts");
 
 __host__ __device__ constexpr int up4(int x) { return (x + 3) & ~3; }
 
@@ -175,10 +178,10 @@ struct RawIds {
 };
 
 // Fill the shared-memory cache of the tile's ids (16-byte loads when aligned),
-// zero the block's scratch and load the placement map.  With `order`, warp 0
-// loads the placement map and orders the experts by (partition, id) -- which
-// needs nothing else -- while the other warps do the rest.  Reads only the
-// caller's inputs.  Ends with a barrier.
+// zero the block's scratch and load the placement map; with `order`, then
+// order the experts by (partition, id) (all warps, expert_order_block, which
+// needs only the placement map).  Reads only the caller's inputs.  Ends with
+// a barrier.
 __device__ void stage_tile(const LayoutArgs& a, const Tile& tl, const Smem& S, RawIds& ids,
                            bool order) {
   const int* src = a.idx + (size_t)tl.t0 * a.topk;
@@ -186,38 +189,35 @@ __device__ void stage_tile(const LayoutArgs& a, const Tile& tl, const Smem& S, R
   ids.s = nullptr;
   const bool cache = tl.n_items <= a.key_cap;
   if (cache) ids.s = S.keys;
-  if (order && warp_id() == 0) {
-    for (int e = lane_id(); e < a.G; e += kWarp) S.part_s[e] = __ldg(a.part_of + e);
-    __syncwarp();
-    expert_order_warp(S.part_s, a.G, a.E, S.pos, S.kcnt);
-  } else {
-    const int r = order ? (int)threadIdx.x - kWarp : (int)threadIdx.x;
-    const int nt = order ? kLThreads - kWarp : kLThreads;
-    if (cache) {
-      const int n = tl.n_items;
-      if ((reinterpret_cast<uintptr_t>(src) & 15) == 0) {
-        const int n4 = n >> 2;
-        const int4* s4 = reinterpret_cast<const int4*>(src);
-        int4* k4 = reinterpret_cast<int4*>(S.keys);
+  const int r = threadIdx.x;
+  if (cache) {
+    const int n = tl.n_items;
+    if ((reinterpret_cast<uintptr_t>(src) & 15) == 0) {
+      const int n4 = n >> 2;
+      const int4* s4 = reinterpret_cast<const int4*>(src);
+      int4* k4 = reinterpret_cast<int4*>(S.keys);
 #pragma unroll 4
-        for (int i = r; i < n4; i += nt) k4[i] = __ldg(s4 + i);
-        for (int i = (n4 << 2) + r; i < n; i += nt) S.keys[i] = __ldg(src + i);
-      } else {
+      for (int i = r; i < n4; i += kLThreads) k4[i] = __ldg(s4 + i);
+      for (int i = (n4 << 2) + r; i < n; i += kLThreads) S.keys[i] = __ldg(src + i);
+    } else {
 #pragma unroll 4
-        for (int i = r; i < n; i += nt) S.keys[i] = __ldg(src + i);
-      }
+      for (int i = r; i < n; i += kLThreads) S.keys[i] = __ldg(src + i);
     }
-    if (!order)
-      for (int e = r; e < a.G; e += nt) S.part_s[e] = __ldg(a.part_of + e);
-    for (int i = r; i < kLWarps * a.G; i += nt) S.whist[i] = 0;
-    for (int i = r; i < a.W; i += nt) S.row[i] = 0;
-    for (int p = r; p < a.E; p += nt) {
-      S.pc[p] = 0;
-      S.pbase[p] = 0;
-    }
-    if (r < 4) S.misc[r] = 0;
   }
+  for (int e = r; e < a.G; e += kLThreads) S.part_s[e] = __ldg(a.part_of + e);
+  for (int i = r; i < kLWarps * a.G; i += kLThreads) S.whist[i] = 0;
+  for (int i = r; i < a.W; i += kLThreads) S.row[i] = 0;
+  for (int p = r; p < a.E; p += kLThreads) {
+    S.pc[p] = 0;
+    S.pbase[p] = 0;
+  }
+  if (r < 4) S.misc[r] = 0;
+  // the expert order's per-(key, chunk) counts live in red (free until the
+  // column sums)
+  if (order)
+    for (int i = r; i < (a.E + 1) * ((a.G + kWarp - 1) / kWarp); i += kLThreads) S.red[i] = 0;
   __syncthreads();
+  if (order) expert_order_block<kLThreads>(S.part_s, a.G, a.E, S.pos, S.red);
 }
 
 __device__ __forceinline__ int item_key(const LayoutArgs& a, const Smem& S, const RawIds& ids,

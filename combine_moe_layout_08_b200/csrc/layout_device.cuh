@@ -62,6 +62,41 @@ __device__ __forceinline__ void expert_order_warp(const int* part_s, int G, int 
   __syncwarp();
 }
 
+// Block-wide version of expert_order_warp: every warp orders 32-expert chunks
+// at once.  The lanes of a chunk holding the same key (partition, or E for an
+// invalid placement) are ranked with a ballot match; an exclusive scan of the
+// per-(key, chunk) counts in key-major order (one warp) gives each (key,
+// chunk) its first position.  wcnt has room for (E + 1) * ceil(G / 32) ints
+// and must be zero on entry.  Reads only part_s[0..G).  Every thread of the
+// block calls it (block barriers inside; pos is complete on return).
+template <int kThreads>
+__device__ __forceinline__ void expert_order_block(const int* part_s, int G, int E, int* pos,
+                                                   int* wcnt) {
+  constexpr int kWarps = kThreads / kWarp;
+  const int lane = lane_id();
+  const int nw = (G + kWarp - 1) / kWarp;
+  const int nbits = key_bits(E + 1);
+  const unsigned lt = lanemask_lt();
+  for (int w = warp_id(); w < nw; w += kWarps) {
+    const int e = w * kWarp + lane;
+    int key = -1;
+    if (e < G) key = valid_part(part_s[e], E) ? part_s[e] : E;
+    const unsigned peers = match_peers(key, nbits);
+    if (e < G) {
+      pos[e] = __popc(peers & lt);  // rank among the chunk's experts of its key
+      if (lane == __ffs(peers) - 1) wcnt[key * nw + w] = __popc(peers);
+    }
+  }
+  __syncthreads();
+  if (warp_id() == 0) (void)warp_exclusive_scan(wcnt, (E + 1) * nw);
+  __syncthreads();
+  for (int e = threadIdx.x; e < G; e += kThreads) {
+    const int key = valid_part(part_s[e], E) ? part_s[e] : E;
+    pos[e] += wcnt[key * nw + e / kWarp];
+  }
+  __syncthreads();
+}
+
 // ---------------------------------------------------------------------------
 // grouped-GEMM tile metadata emitted by the layout kernels themselves
 // (DeepSpeed PR #8180, "Key points": per-tile -> group map from the offsets,
