@@ -322,3 +322,19 @@ def test_python_constants_match_the_header():
                  "MOE_STATUS_BAD_PART", "MOE_STATUS_BAD_ROW", "MOE_STATUS_BAD_COUNT",
                  "MOE_ABI_VERSION"):
         assert eval(defs[name]) == getattr(_lib, name), (name, defs[name])   # integer literals
+
+
+def test_static_scratch_fit_rule(L):
+    """moe_layout_static fits every M when G + (dedup ? E_part : 0) <= 438 (the
+    rule its header states) and not beyond."""
+    cap = 256 * 1024
+
+    def size(G, E, dedup):
+        M = ((1 << 31) - 1) // E                   # the largest batch admitted (M * E_part < 2^31)
+        n = L.moe_layout_workspace_size(ctypes.byref(P(M=M, N=8, G=G, topk=1, E_part=E, dedup=dedup)))
+        assert n > 0
+        return n
+    for G, E, dedup in ((438, 1, 0), (430, 8, 1), (374, 64, 1), (256, 8, 1), (438, 64, 0)):
+        assert size(G, E, dedup) <= cap, (G, E, dedup)
+    for G, E, dedup in ((439, 1, 0), (431, 8, 1), (375, 64, 1)):
+        assert size(G, E, dedup) > cap, (G, E, dedup)
