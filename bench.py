@@ -678,7 +678,8 @@ def run_latency_sweep(args):
     """Decode latency against M on one GPU, in the shape of the Triton-
     distributed issue #117 table (N = 7168, G = 256, topk = 8, bf16,
     M = 2..512): median device time of layout + dispatch (one call, and the
-    separate calls) and of combine, L2 flushed before each step.  Prints one
+    separate calls) and of combine, L2 flushed before each step (the
+    contract line's flush: 256 MiB written, then 256 MiB read).  Prints one
     JSON line; context for the decode path, not the contract line.  Event
     timestamps on this part advance in steps of about 2 us, so single
     intervals of a few us are coarse; medians over many steps are reported.
@@ -694,7 +695,16 @@ def run_latency_sweep(args):
     torch.cuda.set_device(dev)
     base = W.get("decode-M128-uniform")
     stream = torch.cuda.Stream(dev)
+    # the contract line's flush: write then read 256 MiB, so each step starts
+    # with L2 holding clean lines only (no write-backs charged to the step)
     flush_w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    def flush():
+        flush_w.zero_()
+        torch.sum(flush_r, dim=0, out=flush_sink)
+
     rows = []
     for M in SWEEP_M:
         w = dataclasses.replace(base, name=f"decode-M{M}-uniform", M=M)
@@ -727,7 +737,7 @@ def run_latency_sweep(args):
                 t = []
                 for i in range(max(args.warmup, 3) + args.steps):
                     with torch.cuda.stream(stream):
-                        flush_w.zero_()
+                        flush()
                         graph.replay()
                     stream.synchronize()
                     if i >= max(args.warmup, 3):
@@ -743,7 +753,7 @@ def run_latency_sweep(args):
             g_steps, g_flush = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
             with torch.cuda.graph(g_steps, stream=stream):
                 for _ in range(R):
-                    flush_w.zero_()
+                    flush()
                     if separate:
                         buf.layout_(idx, po)
                         buf.dispatch_(d["x"])
@@ -752,7 +762,7 @@ def run_latency_sweep(args):
                     buf.combine_(d["y"], gates)
             with torch.cuda.graph(g_flush, stream=stream):
                 for _ in range(R):
-                    flush_w.zero_()
+                    flush()
 
             def whole(gr, n=max(10, args.steps // 10)):
                 ts = []
