@@ -779,7 +779,30 @@ def run_latency_sweep(args):
             diff = (whole(g_steps) - whole(g_flush)) / R
             g_steps.reset()
             g_flush.reset()
+            # the step alone in a graph, events recorded on the stream around
+            # its replay (after the flush), not inside the graph
+            g_one = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_one, stream=stream):
+                if separate:
+                    buf.layout_(idx, po)
+                    buf.dispatch_(d["x"])
+                else:
+                    buf.layout_dispatch_(idx, po, d["x"])
+                buf.combine_(d["y"], gates)
+            outer = []
+            for i in range(max(args.warmup, 3) + args.steps):
+                e0, e1 = (torch.cuda.Event(enable_timing=True) for _ in range(2))
+                with torch.cuda.stream(stream):
+                    flush()
+                    e0.record()
+                    g_one.replay()
+                    e1.record()
+                e1.synchronize()
+                if i >= max(args.warmup, 3):
+                    outer.append(e0.elapsed_time(e1) * 1e3)
+            g_one.reset()
             key = "separate_" if separate else ""
+            row[key + "step_us_outer_events"] = round(float(np.median(outer)), 2)
             row[key + "step_us_between_flushes"] = round(diff, 2)
             row[key + "step_us"] = round(float(med[0][0]), 2)
             row[key + "layout_dispatch_us"] = round(float(med[1][1]), 2)
@@ -788,6 +811,8 @@ def run_latency_sweep(args):
         rows.append(row)
     print(json.dumps({"metric": "decode latency against M (us, median, L2 flushed)",
                       "note": "step_us: median of one graph replay with events at its ends; "
+                              "step_us_outer_events: median, events recorded on the stream "
+                              "around the replay of a graph holding only the step; "
                               "step_us_between_flushes: the step's share of R back-to-back "
                               "[flush, step] replays (no event node inside the graph)",
                       "config": {"N": base.N, "G": base.G, "topk": base.topk,

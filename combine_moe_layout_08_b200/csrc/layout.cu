@@ -192,16 +192,33 @@ __device__ void stage_tile(const LayoutArgs& a, const Tile& tl, const Smem& S, R
   const int r = threadIdx.x;
   if (cache) {
     const int n = tl.n_items;
+    // batches of 4 predicated loads per thread, all in flight before the
+    // first shared-memory store
+    constexpr int B = 4;
     if ((reinterpret_cast<uintptr_t>(src) & 15) == 0) {
       const int n4 = n >> 2;
       const int4* s4 = reinterpret_cast<const int4*>(src);
       int4* k4 = reinterpret_cast<int4*>(S.keys);
-#pragma unroll 4
-      for (int i = r; i < n4; i += kLThreads) k4[i] = __ldg(s4 + i);
+      for (int i0 = r; i0 < n4; i0 += B * kLThreads) {
+        int4 v[B];
+#pragma unroll
+        for (int j = 0; j < B; ++j)
+          if (i0 + j * kLThreads < n4) v[j] = __ldg(s4 + i0 + j * kLThreads);
+#pragma unroll
+        for (int j = 0; j < B; ++j)
+          if (i0 + j * kLThreads < n4) k4[i0 + j * kLThreads] = v[j];
+      }
       for (int i = (n4 << 2) + r; i < n; i += kLThreads) S.keys[i] = __ldg(src + i);
     } else {
-#pragma unroll 4
-      for (int i = r; i < n; i += kLThreads) S.keys[i] = __ldg(src + i);
+      for (int i0 = r; i0 < n; i0 += B * kLThreads) {
+        int v[B];
+#pragma unroll
+        for (int j = 0; j < B; ++j)
+          if (i0 + j * kLThreads < n) v[j] = __ldg(src + i0 + j * kLThreads);
+#pragma unroll
+        for (int j = 0; j < B; ++j)
+          if (i0 + j * kLThreads < n) S.keys[i0 + j * kLThreads] = v[j];
+      }
     }
   }
   for (int e = r; e < a.G; e += kLThreads) S.part_s[e] = __ldg(a.part_of + e);
@@ -235,14 +252,12 @@ __device__ void rank_count(int n, int K, int* whist, int* key_count, KeyOf key_o
   const int lane = lane_id(), warp = warp_id();
   const int seg = (n + kLWarps - 1) / kLWarps;
   const int beg = min(n, warp * seg), end = min(n, beg + seg);
-  const int nbits = key_bits(K);
   int* wh = whist + warp * K;
-  for (int c = beg; c < end; c += kWarp) {
-    const int i = c + lane;
-    const int key = i < end ? key_of(i) : -1;
-    const unsigned peers = match_peers(key, nbits);
-    if (key >= 0 && lane == __ffs(peers) - 1) wh[key] += __popc(peers);
-    __syncwarp();
+  // per-warp counts only (the order inside a segment does not matter
+  // here): shared-memory atomics on the warp's own histogram
+  for (int i = beg + lane; i < end; i += kWarp) {
+    const int key = key_of(i);
+    if (key >= 0) atomicAdd(&wh[key], 1);
   }
   __syncthreads();
   for (int key = threadIdx.x; key < K; key += kLThreads) {
@@ -305,16 +320,29 @@ __device__ __forceinline__ unsigned long long token_mask(const LayoutArgs& a, co
 // The tile's own row: expert counts (and per-warp bases in whist), with
 // dedup its distinct (token, partition) counts, and the invalid-input
 // counters.  Ends with a barrier.
+// per_warp: also leave the per-warp bases of the stable rank in whist (the
+// one-cluster schedule ranks its tile with them); otherwise only the totals
+// are needed, counted with shared-memory atomics.
 __device__ void count_tile(const LayoutArgs& a, const Tile& tl, const Smem& S, const RawIds& ids,
-                           bool first) {
+                           bool first, bool per_warp) {
   const int G = a.G, E = a.E, lane = lane_id();
   const int fcol = G + (a.dedup ? E : 0);
   int bad = 0;
-  rank_count(tl.n_items, G, S.whist, S.row, [&](int i) {
-    const int e = ids(i);
-    bad += (e < 0 || e >= G);
-    return (e >= 0 && e < G && valid_part(S.part_s[e], E)) ? e : -1;
-  });
+  if (per_warp) {
+    rank_count(tl.n_items, G, S.whist, S.row, [&](int i) {
+      const int e = ids(i);
+      bad += (e < 0 || e >= G);
+      return (e >= 0 && e < G && valid_part(S.part_s[e], E)) ? e : -1;
+    });
+  } else {
+    for (int i = threadIdx.x; i < tl.n_items; i += kLThreads) {
+      const int e = ids(i);
+      if (e < 0 || e >= G)
+        ++bad;
+      else if (valid_part(S.part_s[e], E))
+        atomicAdd(&S.row[e], 1);
+    }
+  }
   int badp = 0;
   if (first)
     for (int e = threadIdx.x; e < G; e += kLThreads) badp += !valid_part(S.part_s[e], E);
@@ -478,7 +506,7 @@ __global__ void __launch_bounds__(kLThreads, kLMinBlocks) layout_cluster_kernel(
   pdl_trigger();
   RawIds ids;
   stage_tile(a, tl, S, ids, true);
-  count_tile(a, tl, S, ids, r == 0);
+  count_tile(a, tl, S, ids, r == 0, true);
   cluster.sync();
 
   // exchange: totals over the cluster and the prefix of the tiles before r
@@ -519,29 +547,41 @@ __global__ void __launch_bounds__(kLThreads, kLMinBlocks) layout_count_kernel(La
   pdl_trigger();
   RawIds ids;
   stage_tile(a, tl, S, ids, false);
-  count_tile(a, tl, S, ids, b == 0);
+  count_tile(a, tl, S, ids, b == 0, false);
   int4* dst = reinterpret_cast<int4*>(a.tile_rows + (size_t)b * a.W);
   const int4* src = reinterpret_cast<const int4*>(S.row);
   for (int i = threadIdx.x; i < (a.W >> 2); i += kLThreads) dst[i] = src[i];
 }
 
 // Column sums of the [rows][W] tile rows in global memory (L2): total over
-// all rows and over rows < b, with up to 8 16-byte loads in flight per
-// thread.  W is a multiple of 4 and at most kRedW.
+// all rows and over rows < b.  Thread slot (c4, s) sums columns 4*c4 .. +3
+// over rows s, s + S, ... with 16-byte loads in batches of 8 rows, all
+// issued (predicated) before any is used -- a rolled loop would wait out one
+// L2 round trip per row; the S partial sums of each column are then added in
+// shared memory.  W is a multiple of 4 and at most kRedW.
 __device__ void column_sums(const int* src, int rows, int W, int b, int* red, int* total,
                             int* before) {
+  constexpr int B = 8;
   const int tid = threadIdx.x;
   const int C4 = W >> 2;
   const int S = C4 <= kLThreads ? kLThreads / C4 : 1;
   for (int slot = tid; slot < C4 * S; slot += kLThreads) {
     const int c4 = slot % C4, s = slot / C4;
     int4 all = make_int4(0, 0, 0, 0), bef = all;
-#pragma unroll 8
-    for (int r = s; r < rows; r += S) {
-      const int4 v = __ldcg(reinterpret_cast<const int4*>(src + (size_t)r * W) + c4);
-      all.x += v.x; all.y += v.y; all.z += v.z; all.w += v.w;
-      if (r < b) {
-        bef.x += v.x; bef.y += v.y; bef.z += v.z; bef.w += v.w;
+    for (int r0 = s; r0 < rows; r0 += B * S) {
+      int4 v[B];
+#pragma unroll
+      for (int j = 0; j < B; ++j) {
+        const int r = r0 + j * S;
+        v[j] = r < rows ? __ldcg(reinterpret_cast<const int4*>(src + (size_t)r * W) + c4)
+                        : make_int4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int j = 0; j < B; ++j) {
+        all.x += v[j].x; all.y += v[j].y; all.z += v[j].z; all.w += v[j].w;
+        if (r0 + j * S < b) {
+          bef.x += v[j].x; bef.y += v[j].y; bef.z += v[j].z; bef.w += v[j].w;
+        }
       }
     }
     const int base = s * W + 4 * c4;

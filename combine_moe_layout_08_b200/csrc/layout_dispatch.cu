@@ -208,7 +208,15 @@ __global__ void __launch_bounds__(kFThreads, 1) layout_dispatch_kernel(FusedArgs
     const int n4 = n_items >> 2;
     const int4* s4 = reinterpret_cast<const int4*>(a.idx);
     int4* k4 = reinterpret_cast<int4*>(ids);
-    for (int i = tid; i < n4; i += kFThreads) k4[i] = __ldg(s4 + i);
+    // two predicated loads per thread in flight together (n4 <= 1024 here)
+    for (int i0 = tid; i0 < n4; i0 += 2 * kFThreads) {
+      const int i1 = i0 + kFThreads;
+      const int4 v0 = __ldg(s4 + i0);
+      int4 v1 = make_int4(0, 0, 0, 0);
+      if (i1 < n4) v1 = __ldg(s4 + i1);
+      k4[i0] = v0;
+      if (i1 < n4) k4[i1] = v1;
+    }
     for (int i = (n4 << 2) + tid; i < n_items; i += kFThreads) ids[i] = __ldg(a.idx + i);
   } else {
     for (int i = tid; i < n_items; i += kFThreads) ids[i] = __ldg(a.idx + i);

@@ -50,3 +50,34 @@ def test_layout_at_the_largest_batch(dedup):
             assert torch.equal(lay.disp_token[t0:t1].long(), want_tok), f"disp_token [{t0}, {t1})"
     del idx, lay, ws
     torch.cuda.empty_cache()
+
+
+# Tiles past the shared-memory id cache (16384 pairs), so ids are read from
+# global memory: 148 tiles of 65504 tokens (topk = 1, every token on expert
+# 0, so each tile counts 65504 for one expert), and one token more, which
+# rounds the tiles up to 65536 tokens and leaves a short last tile.
+# Closed form: exp_row = t.
+@pytest.mark.parametrize("M", [148 * 65504, 148 * 65504 + 1])
+@pytest.mark.parametrize("dedup", [False, True])
+def test_layout_with_tiles_past_the_id_cache(M, dedup):
+    prob = moe.MoEProblem(M, 8, 2, 1, 2, dedup=dedup)
+    idx = torch.zeros((M, 1), dtype=torch.int32, device=DEV)
+    po = torch.tensor([1, 0], dtype=torch.int32, device=DEV)
+    lay = moe.alloc_layout(prob, DEV)
+    lay.status.fill_(-1)
+    ws = torch.empty(moe.layout_workspace_size(prob), dtype=torch.uint8, device=DEV)
+    moe.moe_layout(prob, idx, po, lay, ws)
+    torch.cuda.synchronize()
+    assert lay.status.item() == 0
+    assert lay.expert_count.tolist() == [M, 0]
+    assert lay.expert_offset.tolist() == [0, 0, M]   # expert 1 (partition 0) first
+    assert lay.part_count.tolist() == [0, M] and lay.part_offset.tolist() == [0, 0, M]
+    t = torch.arange(M, dtype=torch.int32, device=DEV)
+    assert torch.equal(lay.exp_row[:M], t)
+    assert torch.equal(lay.disp_token[:M], t)
+    if dedup:                                    # every token in partition 1 only
+        dr = lay.disp_row[:2 * M].view(M, 2)
+        assert bool((dr[:, 0] == -1).all()) and torch.equal(dr[:, 1], t)
+        assert torch.equal(lay.exp_to_disp[:M], t)
+    del idx, lay, ws
+    torch.cuda.empty_cache()
