@@ -296,6 +296,40 @@ def graph_kernel_nodes(graph) -> int:
     return kernels
 
 
+def between_flushes(fns, flush, stream, steps, R=20):
+    """Device time of `fns` per repetition, without event nodes inside it:
+    one graph of R x [flush, fns] minus one of R x [flush], each replay timed
+    whole by events on the stream around it; medians over max(10, steps/10)."""
+    import torch
+    g_work, g_flush = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_work, stream=stream):
+        for _ in range(R):
+            flush()
+            for fn in fns:
+                fn()
+    with torch.cuda.graph(g_flush, stream=stream):
+        for _ in range(R):
+            flush()
+
+    def whole(gr, n=max(10, steps // 10)):
+        ts = []
+        for i in range(n + 3):
+            e0, e1 = (torch.cuda.Event(enable_timing=True) for _ in range(2))
+            with torch.cuda.stream(stream):
+                e0.record()
+                gr.replay()
+                e1.record()
+            e1.synchronize()
+            if i >= 3:
+                ts.append(e0.elapsed_time(e1) * 1e3)
+        return float(np.median(ts))
+
+    us = (whole(g_work) - whole(g_flush)) / R
+    g_work.reset()
+    g_flush.reset()
+    return us
+
+
 def run_ours(args, w):
     import torch
     import torch.distributed as dist
@@ -434,6 +468,11 @@ def run_ours(args, w):
             parts_step()
         per = np.array([parts_step() for _ in range(args.steps)])   # [K, parts] ms
     kern_ms = {name: float(per[:, i].mean()) for i, (name, _) in enumerate(parts)}
+    # the step, and its first part alone, without event nodes inside the
+    # work: R x [flush, work] minus R x [flush], each graph timed as a whole
+    with nvtx("between flushes"):
+        between = {"step": between_flushes([fn for _, fn in parts], flush, stream, args.steps),
+                   parts[0][0]: between_flushes([parts[0][1]], flush, stream, args.steps)}
 
     # end to end through the public API with host buffers
     with nvtx("end to end"):
@@ -478,6 +517,10 @@ def run_ours(args, w):
             "kernels_note": "per-kernel times from a second graph of the step with events "
                             "between its kernels (mean over the same number of steps)",
             "kernels_gbs": {k: round(abytes[k] / (kern_ms[k] * 1e-3) / 1e9, 1) for k in kern_ms},
+            "between_flushes_us": {k: round(v, 2) for k, v in between.items()},
+            "between_flushes_note": "one graph of 20 [flush, work] pairs minus one of 20 flushes, "
+                                    "each timed whole with events outside it, divided by 20 "
+                                    "(median of steps/10 replays): no event node inside the work",
             "algorithmic_bytes_per_step": abytes,
             "roofline": {"bound": "hbm", "kernel": kern_names[dom], "achieved": round(ach, 1),
                          "peak": peak, "unit": "GB/s", "frac": round(ach / peak, 4),
@@ -746,39 +789,13 @@ def run_latency_sweep(args):
                                                                  if inner else (0.0, 0.0)))
                 med.append(np.median(np.array(t), axis=0) * 1e3)
                 graph.reset()
-            # the same step without event nodes inside the graph: R x [flush,
-            # step] minus R x [flush], each timed as a whole (events outside
-            # the graphs), divided by R
-            R = 20
-            g_steps, g_flush = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g_steps, stream=stream):
-                for _ in range(R):
-                    flush()
-                    if separate:
-                        buf.layout_(idx, po)
-                        buf.dispatch_(d["x"])
-                    else:
-                        buf.layout_dispatch_(idx, po, d["x"])
-                    buf.combine_(d["y"], gates)
-            with torch.cuda.graph(g_flush, stream=stream):
-                for _ in range(R):
-                    flush()
-
-            def whole(gr, n=max(10, args.steps // 10)):
-                ts = []
-                for i in range(n + 3):
-                    e0, e1 = (torch.cuda.Event(enable_timing=True) for _ in range(2))
-                    with torch.cuda.stream(stream):
-                        e0.record()
-                        gr.replay()
-                        e1.record()
-                    e1.synchronize()
-                    if i >= 3:
-                        ts.append(e0.elapsed_time(e1) * 1e3)
-                return float(np.median(ts))
-            diff = (whole(g_steps) - whole(g_flush)) / R
-            g_steps.reset()
-            g_flush.reset()
+            # the same step without event nodes inside the graph
+            if separate:
+                work = [lambda: buf.layout_(idx, po), lambda: buf.dispatch_(d["x"])]
+            else:
+                work = [lambda: buf.layout_dispatch_(idx, po, d["x"])]
+            diff = between_flushes(work + [lambda: buf.combine_(d["y"], gates)], flush, stream,
+                                   args.steps)
             # the step alone in a graph, events recorded on the stream around
             # its replay (after the flush), not inside the graph
             g_one = torch.cuda.CUDAGraph()

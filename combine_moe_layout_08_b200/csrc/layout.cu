@@ -317,6 +317,14 @@ __device__ __forceinline__ unsigned long long token_mask(const LayoutArgs& a, co
   return mask;
 }
 
+// The tile's dedup rows [token][partition] kept in shared memory for the
+// inverse map, in the reduction buffer past the tile metadata's expert list
+// (both are free by then), when they fit; nullptr otherwise.
+__device__ __forceinline__ int* tile_drows(const LayoutArgs& a, const Tile& tl, const Smem& S) {
+  const int off = up4(a.G);
+  return (long long)tl.ntok * a.E <= 2 * kRedW - off ? S.red + off : nullptr;
+}
+
 // The tile's own row: expert counts (and per-warp bases in whist), with
 // dedup its distinct (token, partition) counts, and the invalid-input
 // counters.  Ends with a barrier.
@@ -412,6 +420,8 @@ __device__ void rank_tile_parts(const LayoutArgs& a, const Tile& tl, const Smem&
                                 const RawIds& ids) {
   const int E = a.E, lane = lane_id(), warp = warp_id(), tid = threadIdx.x;
   const unsigned lt = lanemask_lt();
+  int* drs = tile_drows(a, tl, S);
+  const bool vec8 = E == 8 && (reinterpret_cast<uintptr_t>(a.disp_row) & 15) == 0;
   for (int r0 = 0; r0 < tl.ntok; r0 += kLThreads) {
     const int t = r0 + tid;
     const unsigned long long mask = t < tl.ntok ? token_mask(a, ids, S.part_s, t) : 0ull;
@@ -431,16 +441,34 @@ __device__ void rank_tile_parts(const LayoutArgs& a, const Tile& tl, const Smem&
     }
     __syncthreads();
     const int tg = tl.t0 + t;
-    for (int p = 0; p < E; ++p) {
-      const bool has = (mask >> p) & 1ull;
-      const unsigned bal = __ballot_sync(kFull, has);
+    auto row_of = [&](int p, bool has, unsigned bal) {
+      int row = -1;
+      if (has) {
+        row = S.poff[p] + S.ppre[p] + S.wp[warp * E + p] + __popc(bal & lt);
+        a.disp_token[row] = tg;
+      }
+      if (drs) drs[t * E + p] = row;
+      return row;
+    };
+    if (vec8) {
+      // eight partitions: the token's rows leave as two 16-byte stores
+      int rr[8];
+#pragma unroll
+      for (int p = 0; p < 8; ++p) {
+        const bool has = (mask >> p) & 1ull;
+        const unsigned bal = __ballot_sync(kFull, has);
+        rr[p] = t < tl.ntok ? row_of(p, has, bal) : -1;
+      }
       if (t < tl.ntok) {
-        int row = -1;
-        if (has) {
-          row = S.poff[p] + S.ppre[p] + S.wp[warp * E + p] + __popc(bal & lt);
-          a.disp_token[row] = tg;
-        }
-        a.disp_row[(size_t)tg * E + p] = row;
+        int4* d = reinterpret_cast<int4*>(a.disp_row + (size_t)tg * 8);
+        d[0] = make_int4(rr[0], rr[1], rr[2], rr[3]);
+        d[1] = make_int4(rr[4], rr[5], rr[6], rr[7]);
+      }
+    } else {
+      for (int p = 0; p < E; ++p) {
+        const bool has = (mask >> p) & 1ull;
+        const unsigned bal = __ballot_sync(kFull, has);
+        if (t < tl.ntok) a.disp_row[(size_t)tg * E + p] = row_of(p, has, bal);
       }
     }
     __syncthreads();
@@ -452,6 +480,7 @@ __device__ void rank_tile_items(const LayoutArgs& a, const Tile& tl, const Smem&
                                 const RawIds& ids) {
   const int G = a.G, E = a.E;
   int* exp_row = a.exp_row + (size_t)tl.t0 * a.topk;
+  const int* drs = a.dedup ? tile_drows(a, tl, S) : nullptr;
   rank_assign(
       tl.n_items, G, S.whist, [&](int i) { return item_key(a, S, ids, i); },
       [&](int i, int e, int r) {
@@ -461,7 +490,8 @@ __device__ void rank_tile_items(const LayoutArgs& a, const Tile& tl, const Smem&
         if (!a.dedup) {
           a.disp_token[row] = t;
         } else {
-          a.exp_to_disp[row] = a.disp_row[(size_t)t * E + S.part_s[e]];
+          a.exp_to_disp[row] = drs ? drs[(i / a.topk) * E + S.part_s[e]]
+                                   : a.disp_row[(size_t)t * E + S.part_s[e]];
         }
       },
       [&](int i) { exp_row[i] = -1; });
