@@ -94,6 +94,7 @@ struct LayoutArgs {
   int n_tiles;  // tiles (= blocks)
   int key_cap;  // ids the shared-memory cache holds (0: read from global)
   int W;        // ints per tile row
+  unsigned topk_magic;  // floor((2^32 - 1) / topk): i / topk without a divide
   const int* __restrict__ idx;
   const int* __restrict__ part_of;
   int* tile_rows;  // [n_tiles][W]   (two-launch schedule)
@@ -190,6 +191,8 @@ __device__ void stage_tile(const LayoutArgs& a, const Tile& tl, const Smem& S, R
   const bool cache = tl.n_items <= a.key_cap;
   if (cache) ids.s = S.keys;
   const int r = threadIdx.x;
+  // the first placement entry of this thread, in flight with the ids
+  const int part0 = r < a.G ? __ldg(a.part_of + r) : 0;
   if (cache) {
     const int n = tl.n_items;
     // batches of 4 predicated loads per thread, all in flight before the
@@ -221,7 +224,8 @@ __device__ void stage_tile(const LayoutArgs& a, const Tile& tl, const Smem& S, R
       }
     }
   }
-  for (int e = r; e < a.G; e += kLThreads) S.part_s[e] = __ldg(a.part_of + e);
+  if (r < a.G) S.part_s[r] = part0;
+  for (int e = r + kLThreads; e < a.G; e += kLThreads) S.part_s[e] = __ldg(a.part_of + e);
   for (int i = r; i < kLWarps * a.G; i += kLThreads) S.whist[i] = 0;
   for (int i = r; i < a.W; i += kLThreads) S.row[i] = 0;
   for (int p = r; p < a.E; p += kLThreads) {
@@ -475,6 +479,15 @@ __device__ void rank_tile_parts(const LayoutArgs& a, const Tile& tl, const Smem&
   }
 }
 
+// i / topk for 0 <= i < 2^31: the high product with floor((2^32 - 1) / topk)
+// is at most one below the quotient (its error is below 2i / 2^32 < 1), and
+// one correction step makes it exact.
+__device__ __forceinline__ int div_topk(const LayoutArgs& a, int i) {
+  unsigned q = __umulhi((unsigned)i, a.topk_magic);
+  if ((unsigned)i - q * (unsigned)a.topk >= (unsigned)a.topk) ++q;
+  return (int)q;
+}
+
 // expert row of every pair of the tile (second pass of the stable rank)
 __device__ void rank_tile_items(const LayoutArgs& a, const Tile& tl, const Smem& S,
                                 const RawIds& ids) {
@@ -486,11 +499,12 @@ __device__ void rank_tile_items(const LayoutArgs& a, const Tile& tl, const Smem&
       [&](int i, int e, int r) {
         const int row = S.eoff[e] + S.pre[e] + r;
         exp_row[i] = row;
-        const int t = tl.t0 + i / a.topk;
+        const int tk = div_topk(a, i);
+        const int t = tl.t0 + tk;
         if (!a.dedup) {
           a.disp_token[row] = t;
         } else {
-          a.exp_to_disp[row] = drs ? drs[(i / a.topk) * E + S.part_s[e]]
+          a.exp_to_disp[row] = drs ? drs[tk * E + S.part_s[e]]
                                    : a.disp_row[(size_t)t * E + S.part_s[e]];
         }
       },
@@ -695,6 +709,7 @@ cudaError_t launch_layout(const moe_problem_t& p, const int32_t* topk_idx,
   a.E = p.E_part;
   a.dedup = p.dedup;
   a.W = row_width(p.G, p.E_part, p.dedup);
+  a.topk_magic = 0xffffffffu / (unsigned)p.topk;
   a.idx = topk_idx;
   a.part_of = part_of;
   a.expert_count = lay.expert_count;

@@ -203,7 +203,9 @@ __global__ void __launch_bounds__(kFThreads, 1) layout_dispatch_kernel(FusedArgs
     }
   }
 
-  // 2. every routing id and the placement map; zeroed histogram and flags
+  // 2. every routing id and the placement map (each thread's first entry
+  // in flight with its ids); zeroed histogram and flags
+  const int part0 = tid < G ? __ldg(a.part_of + tid) : 0;
   if ((reinterpret_cast<uintptr_t>(a.idx) & 15) == 0) {
     const int n4 = n_items >> 2;
     const int4* s4 = reinterpret_cast<const int4*>(a.idx);
@@ -222,7 +224,7 @@ __global__ void __launch_bounds__(kFThreads, 1) layout_dispatch_kernel(FusedArgs
     for (int i = tid; i < n_items; i += kFThreads) ids[i] = __ldg(a.idx + i);
   }
   for (int e = tid; e < G; e += kFThreads) {
-    part_s[e] = __ldg(a.part_of + e);
+    part_s[e] = e == tid ? part0 : __ldg(a.part_of + e);
     hist[e] = 0;
   }
   if (tid < 4) misc[tid] = 0;
