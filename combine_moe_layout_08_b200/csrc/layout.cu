@@ -321,9 +321,10 @@ __device__ __forceinline__ unsigned long long token_mask(const LayoutArgs& a, co
   return mask;
 }
 
-// The tile's dedup rows [token][partition] kept in shared memory for the
-// inverse map, in the reduction buffer past the tile metadata's expert list
-// (both are free by then), when they fit; nullptr otherwise.
+// Where the tile's dedup rows [token][partition] are kept in shared memory
+// for the inverse map: the reduction buffer (free once the column sums are
+// done), past the G ints that the tile metadata's expert list may occupy
+// there; nullptr when ntok * E_part does not fit.
 __device__ __forceinline__ int* tile_drows(const LayoutArgs& a, const Tile& tl, const Smem& S) {
   const int off = up4(a.G);
   return (long long)tl.ntok * a.E <= 2 * kRedW - off ? S.red + off : nullptr;
