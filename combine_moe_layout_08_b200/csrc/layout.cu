@@ -538,7 +538,22 @@ __device__ void write_tiles(const LayoutArgs& a, const Smem& S, int b, int nb) {
 // ---------------------------------------------------------------------------
 // schedule 1: one cluster of gridDim.x blocks
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kLThreads, kLMinBlocks) layout_cluster_kernel(LayoutArgs a) {
+// The layout kernels are instantiated per mode (bit 0: dedup, bit 1:
+// tile metadata), fixed in a local copy of the arguments, so that each
+// instantiation holds only the code its mode runs.  Measured on B200: the
+// denser code (an SM fetches a kernel's instructions afresh at every
+// launch) takes 1.6 us off the M = 4096 layout and 0.7 us off the dedup ones.
+template <int kMode>
+__device__ __forceinline__ LayoutArgs with_mode(const LayoutArgs& in) {
+  LayoutArgs a = in;
+  a.dedup = kMode & 1;
+  if (!(kMode & 2)) a.tiles.block_m = 0;
+  return a;
+}
+
+template <int kMode>
+__global__ void __launch_bounds__(kLThreads, kLMinBlocks) layout_cluster_kernel(LayoutArgs a_in) {
+  const LayoutArgs a = with_mode<kMode>(a_in);
   extern __shared__ __align__(16) int sm[];
   cg::cluster_group cluster = cg::this_cluster();
   const LayoutSmem P(a.G, a.E, a.W, a.key_cap);
@@ -582,19 +597,6 @@ __global__ void __launch_bounds__(kLThreads, kLMinBlocks) layout_cluster_kernel(
 // ---------------------------------------------------------------------------
 // schedule 2: one tile per SM, two launches
 // ---------------------------------------------------------------------------
-// The two-launch kernels are instantiated per mode (bit 0: dedup, bit 1:
-// tile metadata), fixed in a local copy of the arguments, so that each
-// instantiation holds only the code its mode runs.  Measured on B200: the
-// denser code (an SM fetches a kernel's instructions afresh at every
-// launch) takes 1.6 us off the M = 4096 layout and 0.7 us off the dedup ones.
-template <int kMode>
-__device__ __forceinline__ LayoutArgs with_mode(const LayoutArgs& in) {
-  LayoutArgs a = in;
-  a.dedup = kMode & 1;
-  if (!(kMode & 2)) a.tiles.block_m = 0;
-  return a;
-}
-
 template <int kMode>
 __global__ void __launch_bounds__(kLThreads, kLMinBlocks) layout_count_kernel(LayoutArgs a_in) {
   const LayoutArgs a = with_mode<kMode>(a_in);
@@ -765,7 +767,10 @@ cudaError_t launch_layout(const moe_problem_t& p, const int32_t* topk_idx,
     a.key_cap = a.T * p.topk;
     a.tile_rows = nullptr;
     const size_t smem = smem_bytes(p, a.key_cap);
-    cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void*>(layout_cluster_kernel), smem);
+    const int mode = (p.dedup ? 1 : 0) | (tiles.block_m > 0 ? 2 : 0);
+    void (*kernel)(LayoutArgs) = mode == 0 ? layout_cluster_kernel<0> : mode == 1 ? layout_cluster_kernel<1>
+                                 : mode == 2 ? layout_cluster_kernel<2> : layout_cluster_kernel<3>;
+    cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void*>(kernel), smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(C);
@@ -781,7 +786,7 @@ cudaError_t launch_layout(const moe_problem_t& p, const int32_t* topk_idx,
     attr[1].val.programmaticStreamSerializationAllowed = MOE_USE_PDL;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    e = cudaLaunchKernelEx(&cfg, layout_cluster_kernel, a);
+    e = cudaLaunchKernelEx(&cfg, kernel, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }
