@@ -126,7 +126,7 @@ __device__ __forceinline__ Tile tile_of(const LayoutArgs& a, int b) {
 // shared-memory plan (ints, every array 16-byte aligned)
 // ---------------------------------------------------------------------------
 struct LayoutSmem {
-  int part_s, eoff, pos, scanbuf, row, ctot, cpre, red, whist, kcnt, pc, poff, pbase, wp, misc,
+  int part_s, eoff, pos, scanbuf, row, ctot, cpre, red, whist, pc, poff, pbase, wp, misc,
       keys, total;
   __host__ __device__ LayoutSmem(int G, int E, int W, int key_cap) {
     int o = 0;
@@ -139,7 +139,6 @@ struct LayoutSmem {
     cpre = o; o += up4(W);
     red = o; o += 2 * kRedW;
     whist = o; o += up4(kLWarps * G);
-    kcnt = o; o += up4(E + 1);
     pc = o; o += up4(E);
     poff = o; o += up4(E + 1);
     pbase = o; o += up4(E);
@@ -151,14 +150,14 @@ struct LayoutSmem {
 };
 
 struct Smem {
-  int *part_s, *eoff, *pos, *scanbuf, *row, *ctot, *cpre, *red, *whist, *kcnt, *pc, *poff, *pbase,
+  int *part_s, *eoff, *pos, *scanbuf, *row, *ctot, *cpre, *red, *whist, *pc, *poff, *pbase,
       *wp, *misc, *keys;
   // views: totals / tile prefixes per expert and per partition
   int *tot, *pre, *ptot, *ppre;
   __device__ Smem(int* sm, const LayoutSmem& P, int G)
       : part_s(sm + P.part_s), eoff(sm + P.eoff), pos(sm + P.pos), scanbuf(sm + P.scanbuf),
         row(sm + P.row), ctot(sm + P.ctot), cpre(sm + P.cpre), red(sm + P.red),
-        whist(sm + P.whist), kcnt(sm + P.kcnt), pc(sm + P.pc), poff(sm + P.poff),
+        whist(sm + P.whist), pc(sm + P.pc), poff(sm + P.poff),
         pbase(sm + P.pbase), wp(sm + P.wp), misc(sm + P.misc), keys(sm + P.keys) {
     tot = ctot;
     pre = cpre;
@@ -674,7 +673,7 @@ __global__ void __launch_bounds__(kLThreads, kLMinBlocks) layout_rank_kernel(Lay
   const Tile tl = tile_of(a, b);
   // Everything that depends only on the caller's inputs -- which were
   // complete before layout_count_kernel started -- runs before the wait:
-  // the tile's ids, the expert order (warp 0, meanwhile) and the tile's
+  // the tile's ids, the expert order (every warp) and the tile's
   // per-warp counts.
   RawIds ids;
   stage_tile(a, tl, S, ids, true);
