@@ -230,7 +230,8 @@ def run_reference(args, w):
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": "f8e4m3+bf16" if w.fp8 else "bf16",
+        "data": "synthetic",
         "tokens_per_s": round(tokens * args.steps / total, 1),
         "config": config_of(w, extra={"sample_tokens": tokens}),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
